@@ -1,0 +1,138 @@
+"""Pins for the attention oracle: hand-worked cases, closed forms, invariants, brute force and an
+independent library routine. A dropped scale, a wrong softmax axis, a transposed operand or a
+missing max subtraction each fails at least one test here."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth_inputs import normal
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def test_hand_cases(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "attention_hand.json")))
+    for case in g["cases"]:
+        o = oracle.attention(np.array(case["q"]), np.array(case["k"]), np.array(case["v"]), scale=case["scale"])
+        np.testing.assert_allclose(o, np.array(case["o"]), rtol=0, atol=1e-12)
+
+
+def test_rows_sum_to_one():
+    q = normal((3, 17, 40), 5)
+    k = normal((3, 29, 40), 6)
+    p = oracle.softmax_weights(q, k, 1 / math.sqrt(40))
+    np.testing.assert_allclose(p.sum(-1), 1.0, atol=1e-14)
+    assert (p > 0).all()
+
+
+def test_lk1_returns_v():
+    q = normal((2, 3, 5, 8), 1)
+    k = normal((2, 3, 1, 8), 2)
+    v = normal((2, 3, 1, 8), 3)
+    o = oracle.attention(q, k, v)
+    np.testing.assert_allclose(o, np.broadcast_to(v, o.shape), atol=0, rtol=0)
+
+
+def test_equal_scores_mean_of_v():
+    q = np.zeros((1, 2, 4, 16))
+    k = normal((1, 2, 33, 16), 4)
+    v = normal((1, 2, 33, 16), 5).astype(np.float64)
+    o = oracle.attention(q, k, v)
+    np.testing.assert_allclose(o, np.broadcast_to(v.mean(axis=2, keepdims=True), o.shape), atol=1e-14)
+
+
+def test_lk2_sigmoid_closed_form():
+    # two keys: weight of key 1 is the logistic function of scale * q.(k1 - k0)
+    rng = np.random.default_rng(0)
+    q = rng.normal(size=(1, 1, 6, 4))
+    k = rng.normal(size=(1, 1, 2, 4))
+    v = rng.normal(size=(1, 1, 2, 3))
+    scale = 0.37
+    o = oracle.attention(q, k, v, scale=scale)
+    for i in range(6):
+        d = scale * float(q[0, 0, i] @ (k[0, 0, 1] - k[0, 0, 0]))
+        w1 = 1.0 / (1.0 + math.exp(-d))
+        ref = (1 - w1) * v[0, 0, 0] + w1 * v[0, 0, 1]
+        np.testing.assert_allclose(o[0, 0, i], ref, atol=1e-13)
+
+
+def test_large_scores_do_not_overflow():
+    # scores near 1e4: exp without the max subtraction overflows to inf
+    q = np.array([[[[100.0, 0.0]]]])
+    k = np.array([[[[100.0, 0.0], [99.95, 0.0]]]])
+    v = np.array([[[[1.0], [3.0]]]])
+    o = oracle.attention(q, k, v, scale=1.0)
+    w1 = 1.0 / (1.0 + math.exp(100.0 * 100.0 - 100.0 * 99.95))
+    np.testing.assert_allclose(o[0, 0, 0, 0], (1 - w1) * 1.0 + w1 * 3.0, rtol=1e-12)
+
+
+def test_key_shift_invariance_and_value_linearity():
+    q = normal((1, 2, 9, 8), 11).astype(np.float64)
+    k = normal((1, 2, 13, 8), 12).astype(np.float64)
+    v1 = normal((1, 2, 13, 8), 13).astype(np.float64)
+    v2 = normal((1, 2, 13, 8), 14).astype(np.float64)
+    u = normal((8,), 15).astype(np.float64)
+    o = oracle.attention(q, k, v1)
+    np.testing.assert_allclose(oracle.attention(q, k + u, v1), o, atol=1e-12)
+    np.testing.assert_allclose(oracle.attention(q, k, 2.0 * v1 - 3.0 * v2),
+                               2.0 * o - 3.0 * oracle.attention(q, k, v2), atol=1e-12)
+
+
+def test_one_hot_retrieval():
+    # orthonormal keys and q = 30 * k_j: weight of key j is ~1, so the output is ~V_j
+    dh = 16
+    k = np.eye(dh)[None, None]
+    v = normal((1, 1, dh, 5), 21).astype(np.float64)
+    q = 30.0 * k[:, :, [3, 7]] * math.sqrt(dh)
+    o = oracle.attention(q, k, v)
+    np.testing.assert_allclose(o[0, 0, 0], v[0, 0, 3], atol=1e-9)
+    np.testing.assert_allclose(o[0, 0, 1], v[0, 0, 7], atol=1e-9)
+
+
+def test_brute_force_loops():
+    q = normal((2, 1, 3, 4), 31).astype(np.float64)
+    k = normal((2, 1, 5, 4), 32).astype(np.float64)
+    v = normal((2, 1, 5, 4), 33).astype(np.float64)
+    o = oracle.attention(q, k, v, scale=0.5)
+    for b in range(2):
+        for i in range(3):
+            s = [0.5 * sum(q[b, 0, i, d] * k[b, 0, j, d] for d in range(4)) for j in range(5)]
+            e = [math.exp(x) for x in s]
+            z = sum(e)
+            for d in range(4):
+                assert abs(o[b, 0, i, d] - sum(e[j] * v[b, 0, j, d] for j in range(5)) / z) < 1e-12
+
+
+def test_against_torch_sdpa_float64():
+    q = normal((2, 3, 40, 24), 41).astype(np.float64)
+    k = normal((2, 3, 77, 24), 42).astype(np.float64)
+    v = normal((2, 3, 77, 24), 43).astype(np.float64)
+    ref = torch.nn.functional.scaled_dot_product_attention(torch.from_numpy(q), torch.from_numpy(k),
+                                                           torch.from_numpy(v)).numpy()
+    np.testing.assert_allclose(oracle.attention(q, k, v), ref, atol=1e-12)
+
+
+def test_row_subset_and_blocking_agree():
+    q = normal((2, 2, 50, 8), 51)
+    k = normal((2, 2, 40, 8), 52)
+    v = normal((2, 2, 40, 8), 53)
+    full = oracle.attention(q, k, v, row_block=7)
+    np.testing.assert_allclose(full, oracle.attention(q, k, v, row_block=1000), atol=1e-14)
+    rows = np.array([[0, 0, 0], [1, 1, 49], [0, 1, 17], [1, 0, 3]])
+    np.testing.assert_allclose(oracle.attention_rows(q, k, v, rows),
+                               full[rows[:, 0], rows[:, 1], rows[:, 2]], atol=1e-14)
+
+
+def test_bf16_inputs_are_taken_exactly():
+    qf = normal((1, 1, 4, 8), 61)
+    q16 = torch.from_numpy(qf).to(torch.bfloat16)
+    k16 = torch.from_numpy(normal((1, 1, 6, 8), 62)).to(torch.bfloat16)
+    v16 = torch.from_numpy(normal((1, 1, 6, 8), 63)).to(torch.bfloat16)
+    o = oracle.attention(q16, k16, v16)
+    o2 = oracle.attention(q16.double().numpy(), k16.double().numpy(), v16.double().numpy())
+    np.testing.assert_array_equal(o, o2)
