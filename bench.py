@@ -1,0 +1,468 @@
+"""Benchmark of the UNet latent-attention hot path on B200.
+
+One step = one pass of the whole hot path on the SD1.5 512x512 top-level block (B = 2 as the CFG
+pair, 64x64 latent tokens, C = 320, 8 heads of dh = 40):
+    GroupNorm [2,320,64,64] -> self-attention Lq = Lk = 4096 -> cross-attention Lk = 77
+    -> CFG + DDIM update of the [1,4,64,64] latent,
+all four as launches of libsdk.so on one stream. Headline metric: attention TFLOP/s over the step
+(4*B*h*Lq*Lk*dh for self plus cross, true dh, divided by the step's device time); each kernel's
+own TFLOP/s or GB/s and roofline fraction are reported beside it.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (torchrun) every rank runs an independent replica of the step on its own GPU (the
+path has no exchange step): weak scaling, value = all ranks' work / max-over-ranks time.
+``--impl reference`` times the CPU oracle (fp64 numpy) on a bounded sample of the same step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth_inputs as si  # noqa: E402
+
+WID = 2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+ATTN_SOURCES = ["unet_latent_attention_b200/csrc/attention_sm100.cu", "unet_latent_attention_b200/csrc/sm100_ptx.cuh"]
+TRAFFIC_FILE = "profiles/attention_self_sd15_512.md"
+
+
+def workload():
+    w = si.WORKLOADS[WID]
+    attn = dict(w.attention)
+    return w, attn["self"], attn["cross"], w.group_norm[0][1], w.latent
+
+
+def attention_flops(s) -> int:
+    return s.flops
+
+
+def reduce_max(vals, device):
+    """Element-wise max over ranks (identity when torch.distributed is not initialised)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def whole_job_tflops(flops_per_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Weak scaling: every rank runs `steps` steps; the job's time is the slowest rank's."""
+    return flops_per_step * steps * world / (max_ms * 1e-3) / 1e12
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash(paths) -> str:
+    h = hashlib.sha256()
+    for p in paths:
+        h.update(open(os.path.join(ROOT, p), "rb").read())
+    return h.hexdigest()
+
+
+def recorded_traffic():
+    """dram bytes per launch of the self-attention kernel from the committed ncu summary, or None
+    if that summary was taken on a different kernel source."""
+    p = os.path.join(ROOT, TRAFFIC_FILE)
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    for line in open(p):
+        if ":" in line and line.strip().startswith(("source_sha256", "traffic_bytes_per_launch")):
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256") != source_hash(ATTN_SOURCES):
+        return None
+    try:
+        return int(float(vals["traffic_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report no clocks rather than guess
+            self.err = str(e)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------ ours
+def make_sets(dev, n_sets, seed0):
+    import torch
+    _, s_self, s_cross, g, lat = workload()
+    g_ = torch.Generator(device=dev)
+    sets = []
+    for r in range(n_sets):
+        g_.manual_seed(seed0 + r)
+
+        def rn(shape, dtype=torch.float32):
+            return torch.randn(shape, generator=g_, device=dev, dtype=torch.float32).to(dtype)
+
+        bf = torch.bfloat16
+        S = dict(
+            q=rn((s_self.B, s_self.heads, s_self.Lq, s_self.dh), bf),
+            k=rn((s_self.B, s_self.heads, s_self.Lk, s_self.dh), bf),
+            v=rn((s_self.B, s_self.heads, s_self.Lk, s_self.dh), bf),
+            qc=rn((s_cross.B, s_cross.heads, s_cross.Lq, s_cross.dh), bf),
+            kc=rn((s_cross.B, s_cross.heads, s_cross.Lk, s_cross.dh), bf),
+            vc=rn((s_cross.B, s_cross.heads, s_cross.Lk, s_cross.dh), bf),
+            x=rn((g.B, g.C, g.H, g.W)),
+            gamma=1 + 0.1 * rn((g.C,)),
+            beta=0.1 * rn((g.C,)),
+            lat=rn(lat), eu=rn(lat), ec=rn(lat),
+        )
+        S["o"] = torch.empty_like(S["q"])
+        S["oc"] = torch.empty_like(S["qc"])
+        S["y"] = torch.empty_like(S["x"])
+        S["lat_out"] = torch.empty_like(S["lat"])
+        sets.append(S)
+    return sets
+
+
+INPUT_KEYS = ["q", "k", "v", "qc", "kc", "vc", "x", "gamma", "beta", "lat", "eu", "ec"]
+OUTPUT_KEYS = ["o", "oc", "y", "lat_out"]
+
+
+def run_step(sdk, S, g, a_t, a_p, w, events=None):
+    if events:
+        events[0].record()
+    sdk.sd_group_norm(S["x"], S["gamma"], S["beta"], g.groups, g.eps, out=S["y"])
+    if events:
+        events[1].record()
+    sdk.sd_attention(S["q"], S["k"], S["v"], out=S["o"])
+    if events:
+        events[2].record()
+    sdk.sd_attention(S["qc"], S["kc"], S["vc"], out=S["oc"])
+    if events:
+        events[3].record()
+    sdk.sd_cfg_ddim_step(S["lat"], S["eu"], S["ec"], w, a_t, a_p, out=S["lat_out"])
+    if events:
+        events[4].record()
+
+
+def bench_ours(args, rank, world, dev):
+    import torch
+    import unet_latent_attention_b200 as sdk
+    from unet_latent_attention_b200 import build
+    build.build()
+    sdk.lib()
+    wl, s_self, s_cross, g, lat = workload()
+    t, a_t, a_p = sdk.ddim_schedule(20)[0]
+    set_bytes = None
+    sets = make_sets(dev, 1, 1000 * WID + 100 * rank)
+    set_bytes = sum(v.numel() * v.element_size() for v in sets[0].values())
+    n_sets = max(2, math.ceil(2.5 * L2_BYTES / set_bytes))
+    sets += make_sets(dev, n_sets - 1, 1000 * WID + 100 * rank + 1)
+    torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        run_step(sdk, sets[i % n_sets], g, a_t, a_p, wl.guidance)
+    sdk.sd_device_status()
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" in os.environ else dev.index) as clk:
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            run_step(sdk, sets[i % n_sets], g, a_t, a_p, wl.guidance, ev[i])
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+    if world > 1:
+        torch.distributed.barrier()
+    sdk.sd_device_status()
+
+    total_ms = ev[0][0].elapsed_time(ev[-1][4])
+    per_kernel = [0.0] * 4
+    for e in ev:
+        for j in range(4):
+            per_kernel[j] += e[j].elapsed_time(e[j + 1])
+    per_kernel = [x / args.steps for x in per_kernel]  # ms per launch
+    red = reduce_max([total_ms] + per_kernel, dev)
+    total_ms, per_kernel = red[0], red[1:]
+
+    flops_step = attention_flops(s_self) + attention_flops(s_cross)
+    ms_step = total_ms / args.steps
+    value = whole_job_tflops(flops_step, args.steps, world, total_ms)
+    pk, pk_kind = peaks()
+    long_region = total_ms > 1000.0
+    tensor_peak = pk["bf16_tflops_sustained"] if long_region else pk["bf16_tflops"]
+    hbm = pk["hbm_gbs"]
+    gn_bytes = g.bytes
+    lat_n = int(np.prod(lat))
+    ddim_bytes = 16 * lat_n
+    cross_bytes = 2 * (2 * s_cross.B * s_cross.heads * s_cross.Lq * s_cross.dh
+                       + 2 * s_cross.B * s_cross.heads * s_cross.Lk * s_cross.dh)
+    kernels = {
+        "group_norm": {"us": per_kernel[0] * 1e3, "GB/s": gn_bytes / (per_kernel[0] * 1e-3) / 1e9},
+        "self_attention": {"us": per_kernel[1] * 1e3,
+                           "TFLOP/s": attention_flops(s_self) / (per_kernel[1] * 1e-3) / 1e12},
+        "cross_attention": {"us": per_kernel[2] * 1e3,
+                            "TFLOP/s": attention_flops(s_cross) / (per_kernel[2] * 1e-3) / 1e12,
+                            "GB/s": cross_bytes / (per_kernel[2] * 1e-3) / 1e9},
+        "cfg_ddim": {"us": per_kernel[3] * 1e3, "GB/s": ddim_bytes / (per_kernel[3] * 1e-3) / 1e9},
+    }
+    for k in ("group_norm", "cfg_ddim", "cross_attention"):
+        kernels[k]["frac_hbm"] = kernels[k]["GB/s"] / hbm
+    kernels["self_attention"]["frac_tensor"] = kernels["self_attention"]["TFLOP/s"] / tensor_peak
+    achieved = kernels["self_attention"]["TFLOP/s"]
+    traffic = recorded_traffic()
+    roofline = {"kernel": "self_attention", "bound": "tensor", "achieved": achieved, "peak": tensor_peak,
+                "unit": "TFLOP/s", "frac": achieved / tensor_peak, "traffic": traffic,
+                "peak_source": f"{pk_kind} bf16 {'sustained' if long_region else 'burst'} (MEASURED_PEAKS.json)"
+                if pk_kind == "measured" else "fallback 1.59 PF burst / 1.4 PF sustained",
+                "algorithmic_flops_per_launch": attention_flops(s_self)}
+
+    e2e = bench_e2e(args, sdk, sets[0], g, a_t, a_p, wl.guidance, flops_step, world, dev)
+    out = {
+        "metric": "attention TFLOP/s over the UNet hot-path step (GroupNorm + self-attn + cross-attn + CFG/DDIM)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "dtypes": {"attention": "bf16 in, fp32 accumulate", "group_norm": "fp32", "cfg_ddim": "fp32"},
+        "data": "synthetic (seeded torch.randn on device, N(0,1); gamma = 1 + 0.1 N, beta = 0.1 N)",
+        "config": {"workload": wl.name + ": B=2 (CFG pair), Lq=4096 (64x64), C=320, 8 heads dh=40, self Lk=4096, "
+                   "cross Lk=77, GroupNorm [2,320,64,64] 32 groups, CFG(w=7.5)+DDIM on [1,4,64,64]",
+                   "B": 2, "heads": 8, "Lq": 4096, "Lk_self": 4096, "Lk_cross": 77, "dh": 40,
+                   "parallelism": f"replicas x{world}",
+                   "l2": f"inputs rotate over {n_sets} sets of {set_bytes / 2**20:.1f} MiB "
+                         f"({n_sets * set_bytes / 2**20:.0f} MiB > 2x L2)"},
+        "kernels": kernels,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+        "host_wall_s_timed_region": wall,
+    }
+    return out, sets
+
+
+def bench_e2e(args, sdk, S, g, a_t, a_p, w, flops_step, world, dev):
+    """Same step through the public API with host buffers: pinned H2D of every input, the four
+    launches, D2H of every output, all inside the timed region."""
+    import torch
+    host_in = {k: S[k].cpu().pin_memory() for k in INPUT_KEYS}
+    host_out = {k: torch.empty(S[k].shape, dtype=S[k].dtype, pin_memory=True) for k in OUTPUT_KEYS}
+    dev_buf = {k: torch.empty_like(S[k]) for k in INPUT_KEYS + OUTPUT_KEYS}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    n = max(3, min(args.steps, 50))
+
+    def one():
+        for k in INPUT_KEYS:
+            dev_buf[k].copy_(host_in[k], non_blocking=True)
+        run_step(sdk, dev_buf, g, a_t, a_p, w)
+        for k in OUTPUT_KEYS:
+            host_out[k].copy_(dev_buf[k], non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = reduce_max([e0.elapsed_time(e1)], dev)[0]
+    return {"value": whole_job_tflops(flops_step, n, world, ms), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms / n, "steps": n}
+
+
+# -------------------------------------------------------------------------------- CPU oracle arm
+_ORACLE_INPUTS = {}
+
+
+def _oracle_inputs():
+    if not _ORACLE_INPUTS:
+        _, s_self, s_cross, g, lat = workload()
+        _ORACLE_INPUTS.update(
+            self=si.attention_qkv(WID, s_self), cross=si.attention_qkv(WID, s_cross, sub=1),
+            gn=si.group_norm_inputs(WID, g), lat=si.latent_inputs(WID, lat))
+    return _ORACLE_INPUTS
+
+
+def oracle_sample(rows_per_head: int, seed: int = 0):
+    """One bounded sample of the step for the CPU oracle: `rows_per_head` query rows of every head
+    for self- and cross-attention, the whole GroupNorm and the whole CFG+DDIM update.
+    Returns (attention seconds, GroupNorm + DDIM seconds, fraction of attention rows computed)."""
+    import oracle
+    wl, s_self, s_cross, g, lat = workload()
+    inp = _oracle_inputs()
+    rng = np.random.default_rng(seed)
+    rows = np.array([[b, h, i] for b in range(s_self.B) for h in range(s_self.heads)
+                     for i in rng.choice(s_self.Lq, rows_per_head, replace=False)])
+    t0 = time.perf_counter()
+    oracle.attention_rows(*inp["self"], rows)
+    oracle.attention_rows(*inp["cross"], rows)
+    t1 = time.perf_counter()
+    oracle.group_norm(*inp["gn"], g.groups, g.eps)
+    oracle.cfg_ddim_step(*inp["lat"], wl.guidance, 0.5, 0.6)
+    t2 = time.perf_counter()
+    frac = rows.shape[0] / (s_self.B * s_self.heads * s_self.Lq)
+    return t1 - t0, t2 - t1, frac
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max((d.get("num_threads", 1) for d in threadpool_info()), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(budget_s: float):
+    """The oracle as it stands, on a row sample calibrated to take about budget_s."""
+    _, s_self, s_cross, _, _ = workload()
+    flops = attention_flops(s_self) + attention_flops(s_cross)
+    rows = 4
+    ta, tg, frac = oracle_sample(rows)
+    while ta + tg < 0.4 * budget_s and rows < 4096:
+        rows = min(4096, int(rows * max(2.0, 0.8 * budget_s / max(ta + tg, 1e-3))))
+        ta, tg, frac = oracle_sample(rows)
+    full_step_s = ta / frac + tg
+    return {"value": flops / full_step_s / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows} query rows per head (of 4096) of self- and cross-attention for all 16 heads "
+                      f"({ta:.2f} s, scaled by the row fraction {frac:.4f}) plus the whole GroupNorm and CFG+DDIM "
+                      f"({tg:.2f} s), fp64 numpy",
+            "seconds": ta + tg, "full_step_s_estimate": full_step_s}
+
+
+def bench_reference(args):
+    """The CPU oracle as the reference arm: each step is a bounded row sample of the same step,
+    scaled to the full step by its row fraction (GroupNorm and DDIM are computed whole)."""
+    _, s_self, s_cross, _, _ = workload()
+    flops = attention_flops(s_self) + attention_flops(s_cross)
+    per_step_budget = max(0.05, min(5.0, 150.0 / max(1, args.steps + args.warmup)))
+    rows = 1
+    ta, tg, frac = oracle_sample(rows)
+    while ta + tg < 0.5 * per_step_budget and rows < 4096:
+        rows *= 2
+        ta, tg, frac = oracle_sample(rows)
+    for i in range(args.warmup):
+        oracle_sample(rows, seed=i)
+    times = []
+    for i in range(args.steps):
+        ta, tg, frac = oracle_sample(rows, seed=1000 + i)
+        times.append(ta / frac + tg)
+    step_s = sum(times) / len(times)
+    value = flops / step_s / 1e12
+    return {"impl": "reference", "metric": "attention TFLOP/s over the UNet hot-path step (GroupNorm + self-attn + "
+                                           "cross-attn + CFG/DDIM)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic (synth_inputs: splitmix64 + Box-Muller, N(0,1))",
+            "config": {"workload": si.WORKLOADS[WID].name + ": B=2, Lq=4096, 8 heads dh=40, self Lk=4096, cross "
+                                                            "Lk=77, GroupNorm [2,320,64,64], CFG+DDIM [1,4,64,64]"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "kind": "oracle", "cores": blas_threads(),
+                             "sample": f"per step: {rows} query rows per head of self- and cross-attention "
+                                       f"(scaled by the row fraction {frac:.5f}) plus the whole GroupNorm and "
+                                       f"CFG+DDIM, fp64 numpy"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(bench_reference(args)), flush=True)
+        return
+
+    import torch
+    import datetime
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+    try:
+        out, _ = bench_ours(args, rank, world, dev)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,131 @@
+/*
+ * sd_kernels.h -- C ABI of the latent-diffusion hot-path kernels for NVIDIA B200 (sm_100a).
+ *
+ * Three operations of one UNet denoising step, each an asynchronous launch on a caller stream:
+ *
+ *   sd_group_norm     GroupNorm of an NCHW fp32 activation (the reduction that feeds every UNet
+ *                     block).
+ *   sd_attention      multi-head softmax(Q K^T * scale) V for the spatial-transformer blocks:
+ *                     self-attention (K, V from the latent map, Lk = H*W) and cross-attention
+ *                     (K, V from the projected 77-token text context).
+ *   sd_cfg_ddim_step  classifier-free guidance fused with a deterministic DDIM latent update.
+ *
+ * Sources: "从零实现扩散模型推理引擎：Rust + wgpu 的 GPU 加速图像生成架构" (the Rust + wgpu engine page):
+ * §1 sampling loop, §3.1 GroupNorm reduction, §3.2 flash cross-attention with online softmax, §4
+ * scheduler step(model_output, timestep, sample, eta), §6 step_inplace, §7 CFG loop; and
+ * "本地部署扩散模型架构与底层运行原理深度解析", section 示例说明 (guidance pseudo-code).
+ *
+ * Conventions for every entry point:
+ *  - Pointers named x, y, q, k, v, o, eps_* are DEVICE pointers to contiguous row-major
+ *    tensors owned by the caller; the library never frees, keeps or reallocates them.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). The call
+ *    enqueues work and returns; results are ready when the stream reaches that point.
+ *  - Argument errors are detected on the host, before anything is launched, and returned
+ *    synchronously (SD_ERR_INVALID_ARG, SD_ERR_UNSUPPORTED, SD_ERR_MISALIGNED). A size of zero
+ *    (empty tensor) returns SD_OK without a launch. A failed launch returns SD_ERR_CUDA; the
+ *    CUDA error text is available from sd_last_error().
+ *  - Device-side failures (a bounded wait inside a kernel that gave up) are recorded in a
+ *    per-device status word and reported by sd_device_status(); kernels never trap.
+ *  - Calls are thread-safe; each uses the device that is current on the calling thread.
+ */
+#ifndef SD_KERNELS_H
+#define SD_KERNELS_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sd_status {
+  SD_OK = 0,
+  SD_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad divisibility, partial overlap */
+  SD_ERR_UNSUPPORTED = 2,  /* a size outside what the kernels implement (e.g. head dim)      */
+  SD_ERR_MISALIGNED = 3,   /* a pointer that breaks a documented alignment rule             */
+  SD_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed; see sd_last_error()     */
+  SD_ERR_TIMEOUT = 5       /* a kernel's bounded wait expired (reported by sd_device_status)*/
+} sd_status;
+
+/*
+ * GroupNorm, "从零实现扩散模型推理引擎：Rust + wgpu 的 GPU 加速图像生成架构" §3.1: for each batch b and
+ * group g (channels [g*C/G, (g+1)*C/G), all H*W positions: one contiguous span in NCHW),
+ *   mean = sum/N, var = sum((x-mean)^2)/N (biased), rstd = 1/sqrt(var + eps),
+ *   y[b,c,h,w] = (x[b,c,h,w] - mean) * rstd * gamma[c] + beta[c].
+ *  x, y   : fp32 [B, C, H, W] contiguous. y may equal x exactly (in place); any other overlap
+ *           is SD_ERR_INVALID_ARG.
+ *  gamma, beta : fp32 [C].
+ *  groups : must divide C (SD_ERR_INVALID_ARG otherwise); 32 in Stable Diffusion.
+ *  eps    : > 0 and finite (1e-5 in Stable Diffusion).
+ * Statistics are accumulated in fp32 with a pairwise (Chan et al.) merge. Groups of up to
+ * 131072 elements with H*W % 4 == 0 and 16-byte aligned x and y are read from HBM once (a
+ * thread-block cluster of up to 8 CTAs holds the group in registers); other shapes take a
+ * streaming path of the same single launch that reads x twice. No global scratch is used.
+ */
+sd_status sd_group_norm(const float* x, const float* gamma, const float* beta, float* y,
+                        int64_t B, int64_t C, int64_t H, int64_t W, int64_t groups, float eps,
+                        void* stream);
+
+/*
+ * Attention, "从零实现扩散模型推理引擎：Rust + wgpu 的 GPU 加速图像生成架构" §3.2: for each batch b, head h
+ * and query row i, O[b,h,i,:] = sum_j softmax_j(scale * Q[b,h,i,:] . K[b,h,j,:]) V[b,h,j,:].
+ * The kernel is a flash-style forward pass (tiles of 128 queries x 128 keys, running max and
+ * running sum, normalisation at the end) on the sm_100a tensor cores with fp32 accumulation.
+ *  q      : bf16 [B, heads, Lq, dh] contiguous.
+ *  k, v   : bf16 [B, heads, Lk, dh] contiguous (self-attention: Lk = Lq = H*W;
+ *           cross-attention: Lk = 77 text tokens, already projected to heads x dh).
+ *  o      : bf16 [B, heads, Lq, dh] contiguous; must not overlap q, k or v.
+ *  dh     : one of 40, 64, 80, 160 (SD1.5 and SDXL head sizes); others are SD_ERR_UNSUPPORTED.
+ *  scale  : finite; callers normally pass 1/sqrt(dh).
+ *  Lq, Lk : >= 1, any value (ragged tails are masked). B*heads <= 65535.
+ * All four pointers must be 16-byte aligned (SD_ERR_MISALIGNED otherwise).
+ */
+sd_status sd_attention(const void* q, const void* k, const void* v, void* o,
+                       int64_t B, int64_t heads, int64_t Lq, int64_t Lk, int64_t dh, float scale,
+                       void* stream);
+
+/*
+ * Guided DDIM step. Guidance from "从零实现扩散模型推理引擎：Rust + wgpu 的 GPU 加速图像生成架构" §7 and
+ * "本地部署扩散模型架构与底层运行原理深度解析" (示例说明): g = eps_u + w * (eps_c - eps_u), where eps_u and
+ * eps_c are the unconditional and conditional halves of the UNet output (batch order
+ * [uncond, cond]). Sampler step (engine page §1 and §4, DDIM with eta = 0):
+ *   x' = sqrt(alpha_prev) * (x - sqrt(1 - alpha_t) * g) / sqrt(alpha_t) + sqrt(1 - alpha_prev) * g
+ * evaluated as x' = A*x + Bc*g with A = sqrt(alpha_prev/alpha_t) and
+ * Bc = sqrt(1 - alpha_prev) - sqrt(alpha_prev (1 - alpha_t) / alpha_t), both formed in double on
+ * the host; alpha_* are cumulative products (alpha-bar) in (0, 1].
+ *  x, eps_u, eps_c, x_out : fp32, n elements each. x_out may equal x (the engine's in-place
+ *           step); any other overlap of x_out with an input is SD_ERR_INVALID_ARG.
+ * Any alignment is accepted; 16-byte aligned pointers take the vectorised path.
+ */
+sd_status sd_cfg_ddim_step(const float* x, const float* eps_u, const float* eps_c, float* x_out,
+                           int64_t n, float w, double alpha_t, double alpha_prev, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* sd_status_string(sd_status status);
+
+/* Detail of the last error returned on the calling thread (static per-thread buffer). */
+const char* sd_last_error(void);
+
+/*
+ * Synchronises `stream`, then reads the current device's status word. Returns SD_ERR_TIMEOUT if
+ * any kernel of this library gave up a bounded wait since the last reset, SD_ERR_CUDA if the
+ * synchronisation failed, SD_OK otherwise. reset != 0 clears the word afterwards.
+ */
+sd_status sd_device_status(void* stream, int reset);
+
+/*
+ * Test hook for the failure path: flags bit 0 makes every later sd_attention launch (any thread,
+ * any device) skip loading its first V tile, so each CTA's bounded wait expires after about one
+ * second, the CTA drains its own copies, frees its tensor memory and returns, and
+ * sd_device_status() reports SD_ERR_TIMEOUT. Outputs of such launches are undefined. flags = 0
+ * restores normal operation. Not for production use.
+ */
+void sd_debug_set_fault(int flags);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int sd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SD_KERNELS_H */

@@ -17,3 +17,28 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return GOLDEN
+
+
+@pytest.fixture(scope="session")
+def cuda():
+    """The CUDA device for -m gpu tests; fails (never skips) when there is none."""
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("this test needs a CUDA device")
+    from unet_latent_attention_b200 import build
+    build.build()
+    return torch.device("cuda:0")
+
+
+def max_abs_mean_abs(a, b):
+    import numpy as np
+    d = np.abs(np.asarray(a, dtype=np.float64) - np.asarray(b, dtype=np.float64))
+    return float(d.max()) if d.size else 0.0, float(d.mean()) if d.size else 0.0
+
+
+def rel_err(gpu, ref):
+    """Norm-wise relative error max|gpu - ref| / max|ref|."""
+    import numpy as np
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.abs(gpu - ref).max() / max(np.abs(ref).max(), 1e-300))

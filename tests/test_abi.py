@@ -1,0 +1,82 @@
+"""Host-side checks that need no GPU: the library builds and loads, exports every function that
+include/sd_kernels.h declares, validates arguments before touching the device, and the binding
+refuses CPU tensors instead of falling back."""
+import ctypes
+
+import pytest
+import torch
+
+import unet_latent_attention_b200 as sdk
+from unet_latent_attention_b200 import build as sdbuild
+
+
+@pytest.fixture(scope="module")
+def L():
+    sdbuild.build()
+    return sdk.lib()
+
+
+def test_exports_every_header_function(L):
+    names = sdk.header_functions()
+    assert {"sd_group_norm", "sd_attention", "sd_cfg_ddim_step", "sd_device_status"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code, name in sdk.STATUS_NAMES.items():
+        assert L.sd_status_string(code).decode() == name
+    assert L.sd_version() >= 100
+
+
+def _err(L):
+    return L.sd_last_error().decode()
+
+
+def test_attention_argument_errors(L):
+    P = 1 << 12  # a 16-byte-aligned dummy address; nothing is launched on these paths
+    assert L.sd_attention(P, P, P, P, 1, 1, 8, 8, 50, 1.0, None) == 2 and "head dim" in _err(L)
+    assert L.sd_attention(P, P, P, P, -1, 1, 8, 8, 40, 1.0, None) == 1
+    assert L.sd_attention(P, P, P, P, 1, 1, 8, 8, 40, float("nan"), None) == 1
+    assert L.sd_attention(P + 2, P, P, P, 1, 1, 8, 8, 40, 1.0, None) == 3
+    assert L.sd_attention(P, P, P, P + 64, 1, 1, 8, 8, 40, 1.0, None) == 1 and "overlap" in _err(L)
+    assert L.sd_attention(0, 0, 0, 0, 0, 8, 8, 8, 40, 1.0, None) == 0  # empty: no launch
+    assert L.sd_attention(0, 0, 0, 0, 1, 1, 4, 0, 40, 1.0, None) == 1  # Lq >= 1 needs a key
+    assert L.sd_attention(P, P, P, P, 70000, 1, 8, 8, 40, 1.0, None) == 2
+
+
+def test_group_norm_argument_errors(L):
+    P = 1 << 12
+    assert L.sd_group_norm(P, P, P, P, 1, 30, 4, 4, 32, 1e-5, None) == 1  # 32 does not divide 30
+    assert L.sd_group_norm(P, P, P, P, 1, 32, 4, 4, 32, 0.0, None) == 1   # eps must be > 0
+    assert L.sd_group_norm(P, P, P, P + 8, 1, 32, 4, 4, 32, 1e-5, None) == 1  # partial overlap
+    assert L.sd_group_norm(0, 0, 0, 0, 0, 32, 4, 4, 32, 1e-5, None) == 0
+
+
+def test_cfg_ddim_argument_errors(L):
+    P = 1 << 12
+    assert L.sd_cfg_ddim_step(P, P + 4096, P + 8192, P, 16, 7.5, 0.0, 0.5, None) == 1  # alpha_t = 0
+    assert L.sd_cfg_ddim_step(P, P + 4096, P + 8192, P, 16, 7.5, 0.5, 1.5, None) == 1  # alpha_prev > 1
+    assert L.sd_cfg_ddim_step(P, P + 4096, P + 8192, P + 4, 16, 7.5, 0.5, 0.6, None) == 1  # partial alias
+    assert L.sd_cfg_ddim_step(P, P + 4096, P + 8192, P + 4096, 16, 7.5, 0.5, 0.6, None) == 1
+    assert L.sd_cfg_ddim_step(0, 0, 0, 0, 0, 7.5, 0.5, 0.6, None) == 0
+
+
+def test_binding_refuses_cpu_tensors(L):
+    q = torch.zeros(1, 1, 8, 40, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        sdk.sd_attention(q, q, q)
+    x = torch.zeros(1, 32, 4, 4)
+    with pytest.raises(ValueError, match="CUDA"):
+        sdk.sd_group_norm(x, torch.ones(32), torch.zeros(32))
+    with pytest.raises(ValueError, match="CUDA"):
+        sdk.sd_cfg_ddim_step(x, x, x, 7.5, 0.5, 0.6)
+
+
+def test_schedule_tables_match_the_oracle():
+    import oracle
+    ours = sdk.ddim_schedule(20)
+    ref = oracle.ddim_schedule(20)
+    assert [t for t, _, _ in ours] == [t for t, _, _ in ref]
+    for (_, a, p), (_, ra, rp) in zip(ours, ref):
+        assert abs(a - ra) < 1e-13 and abs(p - rp) < 1e-13

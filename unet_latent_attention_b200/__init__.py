@@ -1,0 +1,164 @@
+"""Python binding of the sm_100a latent-diffusion hot-path library (``libsdk.so``).
+
+Argument marshalling only: every step runs in the CUDA kernels behind the C ABI declared in
+``include/sd_kernels.h``. PyTorch supplies device memory and the current CUDA stream. There is no
+CPU fallback: if the library is missing or the tensors are not on a CUDA device, the calls raise.
+
+    sd_group_norm(x, gamma, beta, groups=32, eps=1e-5, out=None)
+    sd_attention(q, k, v, scale=None, out=None)
+    sd_cfg_ddim_step(x, eps_u, eps_c, w, alpha_t, alpha_prev, out=None)
+    sd_cfg_ddim_step_from_noise_pred(x, noise_pred, w, alpha_t, alpha_prev, out=None)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+from .schedule import ddim_schedule, scaled_linear_alphas_cumprod  # noqa: F401  (host-side tables)
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsdk.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "sd_kernels.h")
+
+SD_OK = 0
+STATUS_NAMES = {0: "SD_OK", 1: "SD_ERR_INVALID_ARG", 2: "SD_ERR_UNSUPPORTED", 3: "SD_ERR_MISALIGNED",
+                4: "SD_ERR_CUDA", 5: "SD_ERR_TIMEOUT"}
+
+
+class SDError(RuntimeError):
+    """A non-zero sd_status from the library."""
+
+    def __init__(self, func: str, status: int, detail: str):
+        self.status = status
+        super().__init__(f"{func}: {STATUS_NAMES.get(status, status)}: {detail}")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsdk.so once (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m unet_latent_attention_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        i64, f32, f64, vp, c_int = ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_void_p, ctypes.c_int
+        L.sd_group_norm.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
+        L.sd_attention.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
+        L.sd_cfg_ddim_step.argtypes = [vp, vp, vp, vp, i64, f32, f64, f64, vp]
+        L.sd_device_status.argtypes = [vp, c_int]
+        L.sd_debug_set_fault.argtypes = [c_int]
+        L.sd_debug_set_fault.restype = None
+        for f in ("sd_group_norm", "sd_attention", "sd_cfg_ddim_step", "sd_device_status"):
+            getattr(L, f).restype = c_int
+        L.sd_status_string.argtypes = [c_int]
+        L.sd_status_string.restype = ctypes.c_char_p
+        L.sd_last_error.argtypes = []
+        L.sd_last_error.restype = ctypes.c_char_p
+        L.sd_version.restype = c_int
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions that include/sd_kernels.h declares."""
+    text = open(HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sd_[a-z_0-9]+)\s*\(", text)))
+
+
+def _check(func: str, status: int) -> None:
+    if status != SD_OK:
+        raise SDError(func, status, lib().sd_last_error().decode(errors="replace"))
+
+
+def _stream(t) -> int:
+    import torch
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _require_cuda(*ts) -> None:
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError("sd kernels run on CUDA tensors only (no CPU fallback)")
+        if not t.is_contiguous():
+            raise ValueError("sd kernels take contiguous tensors")
+
+
+def sd_group_norm(x, gamma, beta, groups: int = 32, eps: float = 1e-5, out=None):
+    """GroupNorm of fp32 NCHW ``x`` with per-channel ``gamma``/``beta``; ``out`` may be ``x``."""
+    import torch
+    if x.dtype != torch.float32 or gamma.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise ValueError("sd_group_norm takes fp32 tensors")
+    if x.dim() != 4:
+        raise ValueError("x must be [B, C, H, W]")
+    if out is None:
+        out = torch.empty_like(x)
+    _require_cuda(x, gamma, beta, out)
+    B, C, H, W = x.shape
+    if gamma.numel() != C or beta.numel() != C or out.shape != x.shape:
+        raise ValueError("gamma/beta must have C elements and out the shape of x")
+    _check("sd_group_norm", lib().sd_group_norm(x.data_ptr(), gamma.data_ptr(), beta.data_ptr(), out.data_ptr(),
+                                                B, C, H, W, groups, eps, _stream(x)))
+    return out
+
+
+def sd_attention(q, k, v, scale: float | None = None, out=None):
+    """softmax(q k^T * scale) v for bf16 q [B,h,Lq,dh], k/v [B,h,Lk,dh]; scale defaults to 1/sqrt(dh)."""
+    import torch
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise ValueError("sd_attention takes bf16 q, k, v")
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, heads, L, dh]")
+    B, Hh, Lq, dh = q.shape
+    if k.shape[:2] != (B, Hh) or v.shape != k.shape or k.shape[3] != dh:
+        raise ValueError("k and v must be [B, heads, Lk, dh] matching q")
+    if out is None:
+        out = torch.empty_like(q)
+    _require_cuda(q, k, v, out)
+    if out.shape != q.shape or out.dtype != torch.bfloat16:
+        raise ValueError("out must be bf16 with the shape of q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(dh)
+    _check("sd_attention", lib().sd_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hh, Lq,
+                                              k.shape[2], dh, scale, _stream(q)))
+    return out
+
+
+def sd_cfg_ddim_step(x, eps_u, eps_c, w: float, alpha_t: float, alpha_prev: float, out=None):
+    """x' = DDIM(eta=0) step of fp32 latent x with guided noise eps_u + w (eps_c - eps_u); out may be x."""
+    import torch
+    for t in (x, eps_u, eps_c):
+        if t.dtype != torch.float32:
+            raise ValueError("sd_cfg_ddim_step takes fp32 tensors")
+    if eps_u.shape != x.shape or eps_c.shape != x.shape:
+        raise ValueError("eps_u and eps_c must have the shape of x")
+    if out is None:
+        out = torch.empty_like(x)
+    _require_cuda(x, eps_u, eps_c, out)
+    _check("sd_cfg_ddim_step", lib().sd_cfg_ddim_step(x.data_ptr(), eps_u.data_ptr(), eps_c.data_ptr(),
+                                                      out.data_ptr(), x.numel(), w, alpha_t, alpha_prev,
+                                                      _stream(x)))
+    return out
+
+
+def sd_cfg_ddim_step_from_noise_pred(x, noise_pred, w: float, alpha_t: float, alpha_prev: float, out=None):
+    """Same step taking the UNet output for the batch [uncond, cond] (uncond half first)."""
+    eps_u, eps_c = noise_pred.chunk(2, dim=0)
+    return sd_cfg_ddim_step(x, eps_u, eps_c, w, alpha_t, alpha_prev, out=out)
+
+
+def sd_device_status(stream=None, reset: bool = True) -> int:
+    """Synchronise and read the device status word; raises SDError on a recorded device failure."""
+    s = stream.cuda_stream if stream is not None else 0
+    st = lib().sd_device_status(s, 1 if reset else 0)
+    _check("sd_device_status", st)
+    return st
+
+
+def sd_debug_set_fault(flags: int) -> None:
+    """Test hook: bit 0 makes attention launches skip their first V tile (the bounded wait expires)."""
+    lib().sd_debug_set_fault(int(flags))

@@ -1,0 +1,301 @@
+// GroupNorm over NCHW fp32 (sd_group_norm).
+//
+// "从零实现扩散模型推理引擎：Rust + wgpu 的 GPU 加速图像生成架构" §3.1 reduces a group to its sum and sum of
+// squares with a 256-wide workgroup tree, then mean = sum/N, var = sumsq/N - mean^2 (biased) and
+// inv_std = 1/sqrt(var + eps); the page elides the normalise/affine tail. Here:
+//
+//  * A group (C/G channels x H*W, one contiguous span in NCHW) is split over a thread-block
+//    cluster of up to 8 CTAs. Each thread loads its part of the group into registers with 16-byte
+//    streaming loads, so HBM is read exactly once (the resident path).
+//  * Statistics stay in fp32 but are merged as (count, mean, M2) triples with the pairwise update
+//    of Chan, Golub and LeVeque (1979) -- warp shuffles, then shared memory across warps, then
+//    distributed shared memory across the cluster -- instead of sum / sum-of-squares, which
+//    cancels when |mean| >> std. Every CTA of a cluster merges the per-CTA triples in rank order,
+//    so all of them obtain bit-identical statistics.
+//  * The tail is fused: y = x * a_c + b_c with a_c = rstd * gamma[c], b_c = beta[c] - mean * a_c.
+//
+// Shapes the resident path cannot hold (groups above 8 x 16384 elements, H*W not a multiple of 4,
+// pointers not 16-byte aligned) take the streaming path: the same cluster merge, but each CTA
+// sweeps its part twice (statistics, then normalise), so x is read twice (the second time mostly
+// from L2). Neither path uses global scratch memory.
+#include <cooperative_groups.h>
+
+#include <cmath>
+
+#include "sd_internal.h"
+
+namespace cg = cooperative_groups;
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxCluster = 8;
+constexpr int kMaxItems = 16;  // float4 per thread on the resident path
+constexpr int64_t kResidentCap = static_cast<int64_t>(kThreads) * 4 * kMaxItems;  // elements per CTA
+
+struct Stats {
+  float n, mean, m2;
+};
+
+// Chan et al. pairwise merge of two (count, mean, sum of squared deviations) triples.
+__device__ __forceinline__ Stats merge(Stats a, Stats b) {
+  const float n = a.n + b.n;
+  if (n == 0.f) return a;
+  const float d = b.mean - a.mean;
+  const float fb = b.n / n;
+  return Stats{n, fmaf(d, fb, a.mean), a.m2 + b.m2 + d * d * a.n * fb};
+}
+
+__device__ __forceinline__ Stats shfl_down(Stats s, int off) {
+  return Stats{__shfl_down_sync(0xffffffffu, s.n, off), __shfl_down_sync(0xffffffffu, s.mean, off),
+               __shfl_down_sync(0xffffffffu, s.m2, off)};
+}
+
+// Exact statistics of four values (two sweeps over registers).
+__device__ __forceinline__ Stats stats4(float4 v, float n) {
+  if (n == 0.f) return Stats{0.f, 0.f, 0.f};
+  const float mean = (v.x + v.y + v.z + v.w) * 0.25f;
+  const float a = v.x - mean, b = v.y - mean, c = v.z - mean, d = v.w - mean;
+  return Stats{4.f, mean, a * a + b * b + c * c + d * d};
+}
+
+__device__ __forceinline__ float4 ld_stream(const float4* p) {
+  float4 v;
+  asm volatile("ld.global.cs.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void st_stream(float4* p, float4 v) {
+  asm volatile("st.global.cs.v4.f32 [%0], {%1,%2,%3,%4};" :: "l"(p), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
+// Reduces the thread's triple over the CTA, publishes it to the cluster, and returns (in shared
+// memory) the group's mean and rstd as merged by every CTA in the same order.
+__device__ __forceinline__ void cluster_group_stats(Stats st, float eps, float* s_mean, float* s_rstd,
+                                                    Stats* s_warp, Stats* s_cta) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const Stats o = shfl_down(st, off);
+    if (lane + off < 32) st = merge(st, o);
+  }
+  if (lane == 0) s_warp[warp] = st;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Stats a = s_warp[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) a = merge(a, s_warp[w]);
+    *s_cta = a;
+  }
+  cluster.sync();  // every CTA's triple is now visible to the cluster
+  if (threadIdx.x == 0) {
+    const unsigned cs = cluster.num_blocks();
+    Stats a = *cluster.map_shared_rank(s_cta, 0);
+    for (unsigned r = 1; r < cs; ++r) a = merge(a, *cluster.map_shared_rank(s_cta, r));
+    const float var = a.n > 0.f ? fmaxf(a.m2 / a.n, 0.f) : 0.f;
+    *s_mean = a.mean;
+    *s_rstd = rsqrtf(var + eps);
+  }
+  __syncthreads();
+}
+
+// Resident path: one cluster of `cs` CTAs per (b, g); CTA `rank` owns elements
+// [rank*chunk, (rank+1)*chunk) of the group, chunk a multiple of 4, held in registers.
+template <int ITEMS>
+__global__ void __launch_bounds__(kThreads) gn_resident(const float* x, const float* __restrict__ gamma,
+                                                        const float* __restrict__ beta, float* y,
+                                                        int group_elems, int chunk, int hw, int cpg, int groups,
+                                                        float eps) {
+  __shared__ Stats s_warp[kWarps];
+  __shared__ Stats s_cta;
+  __shared__ float s_mean, s_rstd;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int64_t grp = blockIdx.x / cluster.num_blocks();  // b * groups + g
+  const int g = static_cast<int>(grp % groups);
+  const int64_t base = grp * group_elems + static_cast<int64_t>(rank) * chunk;
+  const float4* xg = reinterpret_cast<const float4*>(x + base);
+  const int n4 = chunk >> 2;
+
+  float4 v[ITEMS];
+#pragma unroll
+  for (int i = 0; i < ITEMS; ++i) {
+    const int idx = threadIdx.x + i * kThreads;
+    v[i] = idx < n4 ? ld_stream(xg + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // Thread triple: exact mean of its values, then M2 about it.
+  float sum = 0.f, cnt = 0.f;
+#pragma unroll
+  for (int i = 0; i < ITEMS; ++i) {
+    if (threadIdx.x + i * kThreads < n4) {
+      sum += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+      cnt += 4.f;
+    }
+  }
+  Stats st{cnt, cnt > 0.f ? sum / cnt : 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < ITEMS; ++i) {
+    if (threadIdx.x + i * kThreads < n4) {
+      const float a = v[i].x - st.mean, b = v[i].y - st.mean, c = v[i].z - st.mean, d = v[i].w - st.mean;
+      st.m2 += a * a + b * b + c * c + d * d;
+    }
+  }
+  cluster_group_stats(st, eps, &s_mean, &s_rstd, s_warp, &s_cta);
+  const float mean = s_mean, rstd = s_rstd;
+
+  float4* yg = reinterpret_cast<float4*>(y + base);
+  const int e0 = rank * chunk;
+#pragma unroll
+  for (int i = 0; i < ITEMS; ++i) {
+    const int idx = threadIdx.x + i * kThreads;
+    if (idx < n4) {
+      const int c = g * cpg + (e0 + idx * 4) / hw;  // hw % 4 == 0: a float4 never straddles channels
+      const float a = rstd * __ldg(gamma + c);
+      const float b = fmaf(-mean, a, __ldg(beta + c));
+      st_stream(yg + idx, make_float4(fmaf(v[i].x, a, b), fmaf(v[i].y, a, b), fmaf(v[i].z, a, b),
+                                      fmaf(v[i].w, a, b)));
+    }
+  }
+  cluster.sync();  // peers read s_cta through distributed shared memory; keep it alive until they are done
+}
+
+// Streaming path: any shape and alignment. CTA `rank` of the cluster owns elements [lo, hi) of the
+// group; sweep 1 builds the triple (exact stats of each run of four values, merged pairwise),
+// sweep 2 normalises.
+__global__ void __launch_bounds__(kThreads) gn_streaming(const float* x, const float* __restrict__ gamma,
+                                                         const float* __restrict__ beta, float* y,
+                                                         int64_t group_elems, int64_t chunk, int64_t hw, int cpg,
+                                                         int groups, float eps) {
+  __shared__ Stats s_warp[kWarps];
+  __shared__ Stats s_cta;
+  __shared__ float s_mean, s_rstd;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int64_t rank = cluster.block_rank();
+  const int64_t grp = blockIdx.x / cluster.num_blocks();
+  const int g = static_cast<int>(grp % groups);
+  const int64_t lo = rank * chunk;
+  const int64_t hi = lo + chunk < group_elems ? lo + chunk : group_elems;
+  const float* xg = x + grp * group_elems;
+  float* yg = y + grp * group_elems;
+
+  Stats st{0.f, 0.f, 0.f};
+  for (int64_t e = lo + 4 * threadIdx.x; e < hi; e += 4 * kThreads) {
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int64_t m = hi - e < 4 ? hi - e : 4;
+    v.x = xg[e];
+    if (m > 1) v.y = xg[e + 1];
+    if (m > 2) v.z = xg[e + 2];
+    if (m > 3) v.w = xg[e + 3];
+    Stats r;
+    if (m == 4) {
+      r = stats4(v, 4.f);
+    } else {  // ragged tail of the part: exact stats of m values
+      float s = v.x + (m > 1 ? v.y : 0.f) + (m > 2 ? v.z : 0.f);
+      const float mu = s / static_cast<float>(m);
+      float q = (v.x - mu) * (v.x - mu);
+      if (m > 1) q += (v.y - mu) * (v.y - mu);
+      if (m > 2) q += (v.z - mu) * (v.z - mu);
+      r = Stats{static_cast<float>(m), mu, q};
+    }
+    st = merge(st, r);
+  }
+  cluster_group_stats(st, eps, &s_mean, &s_rstd, s_warp, &s_cta);
+  const float mean = s_mean, rstd = s_rstd;
+  for (int64_t e = lo + threadIdx.x; e < hi; e += kThreads) {
+    const int c = g * cpg + static_cast<int>(e / hw);
+    const float a = rstd * __ldg(gamma + c);
+    yg[e] = fmaf(xg[e], a, fmaf(-mean, a, __ldg(beta + c)));
+  }
+  cluster.sync();
+}
+
+template <int ITEMS>
+cudaError_t launch_resident(dim3 grid, int cs, cudaStream_t s, const float* x, const float* gamma,
+                            const float* beta, float* y, int group_elems, int chunk, int hw, int cpg, int groups,
+                            float eps) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, gn_resident<ITEMS>, x, gamma, beta, y, group_elems, chunk, hw, cpg, groups, eps);
+}
+
+}  // namespace
+
+extern "C" sd_status sd_group_norm(const float* x, const float* gamma, const float* beta, float* y, int64_t B,
+                                   int64_t C, int64_t H, int64_t W, int64_t groups, float eps, void* stream) {
+  if (B < 0 || C < 0 || H < 0 || W < 0) return sd::fail(SD_ERR_INVALID_ARG, "sd_group_norm: negative size");
+  if (groups <= 0 || (C > 0 && C % groups != 0))
+    return sd::fail(SD_ERR_INVALID_ARG, "sd_group_norm: groups must be positive and divide C");
+  if (!(eps > 0.f) || !std::isfinite(eps)) return sd::fail(SD_ERR_INVALID_ARG, "sd_group_norm: eps must be > 0");
+  if (B == 0 || C == 0 || H == 0 || W == 0) return SD_OK;
+  if (!x || !gamma || !beta || !y) return sd::fail(SD_ERR_INVALID_ARG, "sd_group_norm: null pointer");
+  const int64_t hw = H * W;
+  const int64_t cpg = C / groups;
+  const int64_t group_elems = cpg * hw;
+  const int64_t n_groups = B * groups;
+  if (group_elems > (int64_t(1) << 31) - 1 || n_groups * kMaxCluster > 0x7fffffff)
+    return sd::fail(SD_ERR_UNSUPPORTED, "sd_group_norm: tensor too large");
+  const int64_t bytes = B * C * hw * static_cast<int64_t>(sizeof(float));
+  const int64_t pbytes = C * static_cast<int64_t>(sizeof(float));
+  if ((y != x && sd::overlaps(y, bytes, x, bytes)) || sd::overlaps(y, bytes, gamma, pbytes) ||
+      sd::overlaps(y, bytes, beta, pbytes))
+    return sd::fail(SD_ERR_INVALID_ARG, "sd_group_norm: y overlaps an input (only y == x is allowed)");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // Resident path: the smallest cluster (power of two <= 8) that holds the group in registers and
+  // gives at least two CTAs per SM; chunk must be a multiple of 4 elements.
+  const bool vec_ok = hw % 4 == 0 && sd::aligned16(x) && sd::aligned16(y);
+  int cs = 0;
+  if (vec_ok) {
+    const int64_t want_ctas = 2 * static_cast<int64_t>(sd::sm_count());
+    for (int c = 1; c <= kMaxCluster; c *= 2) {
+      if (group_elems % (4 * c) != 0 || group_elems / c > kResidentCap) continue;
+      cs = c;
+      if (n_groups * c >= want_ctas) break;
+    }
+  }
+  cudaError_t err;
+  if (cs > 0) {
+    const int chunk = static_cast<int>(group_elems / cs);
+    const int need = (chunk / 4 + kThreads - 1) / kThreads;
+    const dim3 grid(static_cast<unsigned>(n_groups * cs));
+    const int ge = static_cast<int>(group_elems), ihw = static_cast<int>(hw), icpg = static_cast<int>(cpg),
+              ig = static_cast<int>(groups);
+#define SD_GN_CASE(N) \
+  if (need <= N) err = launch_resident<N>(grid, cs, s, x, gamma, beta, y, ge, chunk, ihw, icpg, ig, eps); else
+    SD_GN_CASE(1) SD_GN_CASE(2) SD_GN_CASE(3) SD_GN_CASE(4) SD_GN_CASE(5) SD_GN_CASE(6) SD_GN_CASE(8)
+    SD_GN_CASE(10) SD_GN_CASE(12) SD_GN_CASE(16) err = cudaErrorInvalidValue;
+#undef SD_GN_CASE
+  } else {
+    // Streaming path: a cluster of up to 8 CTAs per group, each with at least 1024 elements.
+    int c = 1;
+    while (c < kMaxCluster && group_elems / (2 * c) >= 1024) c *= 2;
+    const int64_t chunk = (group_elems + c - 1) / c;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(n_groups * c));
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = c;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    err = cudaLaunchKernelEx(&cfg, gn_streaming, x, gamma, beta, y, group_elems, chunk, hw,
+                             static_cast<int>(cpg), static_cast<int>(groups), eps);
+  }
+  return sd::cuda_check(err, "sd_group_norm launch");
+}

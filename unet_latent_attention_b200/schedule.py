@@ -1,0 +1,27 @@
+"""Host-side noise-schedule tables for driving sd_cfg_ddim_step over a denoising loop.
+
+Stable Diffusion's "scaled linear" betas: T points evenly spaced between sqrt(beta_start) and
+sqrt(beta_end), squared; alpha_bar_t is the running product of (1 - beta). The sampler of
+"从零实现扩散模型推理引擎：Rust + wgpu 的 GPU 加速图像生成架构" (§4, scheduler holding alphas_cumprod; the
+order-1 solver is DDIM) steps through evenly strided timesteps; alpha_prev = 1 after the last
+step. Plain Python floats (double precision); the kernel receives alpha_t and alpha_prev.
+"""
+from __future__ import annotations
+
+
+def scaled_linear_alphas_cumprod(beta_start: float = 0.00085, beta_end: float = 0.012, T: int = 1000):
+    lo, hi = beta_start ** 0.5, beta_end ** 0.5
+    out, prod = [], 1.0
+    for i in range(T):
+        r = lo + (hi - lo) * i / (T - 1)
+        prod *= 1.0 - r * r
+        out.append(prod)
+    return out
+
+
+def ddim_schedule(steps: int = 20, T: int = 1000, beta_start: float = 0.00085, beta_end: float = 0.012):
+    """[(t, alpha_t, alpha_prev)] for t = (steps-1)*T/steps, ..., T/steps, 0."""
+    ac = scaled_linear_alphas_cumprod(beta_start, beta_end, T)
+    stride = T // steps
+    ts = [stride * i for i in range(steps - 1, -1, -1)]
+    return [(t, ac[t], ac[ts[i + 1]] if i + 1 < len(ts) else 1.0) for i, t in enumerate(ts)]
