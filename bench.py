@@ -107,14 +107,17 @@ class ClockSampler:
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
-    def __init__(self, index: int):
+    def __init__(self, dev):
         self.samples, self.reasons, self.ok = [], 0, False
         self._stop = threading.Event()
         try:
             import pynvml
+            import torch
             pynvml.nvmlInit()
             self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            uuid = str(torch.cuda.get_device_properties(dev).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)  # the GPU this rank runs on, not NVML index 0
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
         except Exception as e:  # NVML missing: report no clocks rather than guess
@@ -221,14 +224,24 @@ def bench_ours(args, rank, world, dev):
         run_step(sdk, sets[i % n_sets], g, a_t, a_p, wl.guidance)
     sdk.sd_device_status()
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    # The K timed steps are captured once into a CUDA graph (kernel launches of the library on the
+    # capture stream, with external timing events between them) and replayed once, so host launch
+    # overhead never starves the GPU and every kernel is timed on its own stream position.
+    ev = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)] for _ in range(args.steps)]
+    graph = torch.cuda.CUDAGraph()
+    cap_stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.graph(graph, stream=cap_stream):
+        for i in range(args.steps):
+            run_step(sdk, sets[i % n_sets], g, a_t, a_p, wl.guidance, ev[i])
+    graph.replay()  # one untimed replay: instantiation and first-touch costs stay out of the timing
+    torch.cuda.synchronize()
+    sdk.sd_device_status()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" in os.environ else dev.index) as clk:
+    with ClockSampler(dev) as clk:
         t0 = time.perf_counter()
-        for i in range(args.steps):
-            run_step(sdk, sets[i % n_sets], g, a_t, a_p, wl.guidance, ev[i])
+        graph.replay()
         torch.cuda.synchronize()
         wall = time.perf_counter() - t0
     if world > 1:

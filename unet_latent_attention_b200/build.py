@@ -34,9 +34,9 @@ def sources():
     return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
 
 
-def _compile(src: str, verbose_ptxas: bool) -> str:
+def _compile(src: str, verbose_ptxas: bool, extra=()) -> str:
     obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
-    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-c", src, "-o", obj]
+    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *extra, "-c", src, "-o", obj]
     if verbose_ptxas:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -47,24 +47,40 @@ def _compile(src: str, verbose_ptxas: bool) -> str:
     return obj
 
 
-def build(verbose_ptxas: bool = False, force: bool = False) -> str:
-    """Compile every ``csrc/*.cu`` and link ``libsdk.so``; returns the library path."""
+def build(verbose_ptxas: bool = False, force: bool = False, defines=(), out: str | None = None) -> str:
+    """Compile every ``csrc/*.cu`` and link ``libsdk.so``; returns the library path.
+
+    ``defines`` (e.g. ``["SD_POLY_PAIRS=2"]``) and ``out`` build a tuning variant of the library
+    under another name; the default build is the product library."""
+    global BUILD
+    lib_path = out or LIB
+    if defines:
+        tag = "_".join(d.replace("=", "") for d in defines)
+        saved, BUILD = BUILD, os.path.join(BUILD, tag)
+        try:
+            return _build(verbose_ptxas, True, [f"-D{d}" for d in defines], lib_path)
+        finally:
+            BUILD = saved
+    return _build(verbose_ptxas, force, [], lib_path)
+
+
+def _build(verbose_ptxas: bool, force: bool, extra, lib_path: str) -> str:
     os.makedirs(BUILD, exist_ok=True)
     srcs = sources()
     deps = srcs + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
     deps.append(os.path.join(INCLUDE, "sd_kernels.h"))
-    if (not force and not verbose_ptxas and os.path.exists(LIB)
-            and os.path.getmtime(LIB) >= max(os.path.getmtime(d) for d in deps)):
-        return LIB
+    if (not force and not verbose_ptxas and os.path.exists(lib_path)
+            and os.path.getmtime(lib_path) >= max(os.path.getmtime(d) for d in deps)):
+        return lib_path
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas), srcs))
-    tmp = LIB + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas, extra), srcs))
+    tmp = lib_path + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lpthread", "-lrt"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib_path)
+    return lib_path
 
 
 if __name__ == "__main__":

@@ -10,16 +10,20 @@
 //    128-byte swizzle, boxes 64 wide in dh) into a ring of STAGES shared-memory stages; rows past
 //    the sequence end and columns past dh are zero-filled by the TMA unit, which pads dh = 40 to
 //    the MMA depth 48 and masks ragged tails for free.
-//  * One thread issues the tensor-core work: S = Q K^T (tcgen05.mma, bf16 in, fp32 accumulate,
-//    M = 128, N = BN, K = 16 per instruction) into tensor memory, then O += P V with P read
-//    straight from tensor memory (the "A in TMEM" form) and V from shared memory (N-major B).
+//  * One thread issues the tensor-core work from an event loop over the query tiles: S = Q K^T
+//    (tcgen05.mma, bf16 in, fp32 accumulate, M = 128, N = BN, K = 16 per instruction) into tensor
+//    memory, O += P V with P read straight from tensor memory (the "A in TMEM" form) and V from
+//    shared memory (N-major B), and l += P * ones (a 16-column MMA against an all-ones tile) for
+//    the softmax row sums, so the sums use exactly the bf16 probabilities that multiply V.
 //  * Four warps per query tile (one TMEM lane quarter each, one thread per row) run the softmax:
-//    tcgen05.ld the S row, row max, exp2 with scale*log2(e) folded into one FMA, row sum, pack to
-//    bf16 and tcgen05.st P over the S columns. The running max is only raised when it grows by
-//    more than 2^8 (lazy rescaling), so most tiles skip the O correction. Normalisation by l is
-//    deferred to the epilogue, which equals the page's per-step form in exact arithmetic.
-//  * Two query tiles per CTA (NQ = 2) share every K/V tile, halving L2->SM traffic, and let one
-//    tile's softmax overlap the other tile's matrix products.
+//    tcgen05.ld the S row and release it (the next S = Q K^T starts at once), row max over
+//    independent 3-input-max chains, exp2 with scale*log2(e) folded into one packed FMA, pack to
+//    bf16 and tcgen05.st P into its own TMEM columns once the previous P V has consumed them. The
+//    running max is only raised when it grows by more than 2^8 (lazy rescaling), so most tiles
+//    skip the O correction; normalisation by l is deferred to the epilogue, which equals the
+//    page's per-step form in exact arithmetic.
+//  * Two query tiles per CTA (NQ = 2) share every K/V tile, halving L2->SM traffic, and keep the
+//    tensor core busy with one tile while the other is in its softmax.
 //  * Every wait on an mbarrier is bounded (about one second); on expiry the CTA records
 //    SD_ERR_TIMEOUT in the device status word, drains its own in-flight copies and MMAs, frees its
 //    tensor memory and returns. Nothing traps.
@@ -27,6 +31,7 @@
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <mutex>
 
@@ -37,33 +42,82 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128;                          // query rows per tile = TMEM lanes
+#ifndef SD_POLY_PAIRS
+#define SD_POLY_PAIRS -1  // tuning override of the per-head-dim choice in the launch table
+#endif
+
+#ifdef SD_TRACE
+// Tuning builds only: per-CTA phase timestamps of the first softmax warp and of the MMA warp.
+constexpr int kTraceCtas = 64, kTraceIters = 40, kTraceSlots = 8;
+__device__ long long g_trace[kTraceCtas][12][kTraceIters][kTraceSlots];
+#define SD_TR(role, j, slot)                                                                        \
+  do {                                                                                              \
+    const int cta_ = blockIdx.x + gridDim.x * blockIdx.y;                                          \
+    if (cta_ < kTraceCtas && (j) < kTraceIters) g_trace[cta_][role][j][slot] = clock64();           \
+  } while (0)
+#else
+#define SD_TR(role, j, slot) \
+  do {                       \
+  } while (0)
+#endif
+
+#ifndef SD_PINGPONG
+#define SD_PINGPONG 1  // alternate the two query tiles' exp2 phases on each SM sub-partition
+#endif
+
+#ifndef SD_STAGES_SMALL
+#define SD_STAGES_SMALL 5  // K/V ring depth for head dims <= 64 (one 16 KB K and V tile per stage)
+#endif
+
+constexpr int BM = 128;                               // query rows per tile = TMEM lanes
 constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at B200 clocks
 
-template <int DHP_, int BN_, int NQ_, int STAGES_>
+// P_SEP: P has its own TMEM columns (else it overwrites S, and the next S waits for P V).
+// L_IN_V: the softmax row sums come out of the P V product itself: a fix-up warp writes bf16 1.0
+//         into column DH of every V tile once it lands (the TMA zero-fills columns >= DH), so O's
+//         column DH accumulates sum_j P_ij with no extra MMA (else fp32 adds in registers).
+template <int DH_, int BN_, int NQ_, int STAGES_, bool P_SEP_, bool L_IN_V_, int POLY_ = 0>
 struct Cfg {
-  static constexpr int DHP = DHP_;        // head dim padded to the MMA granule (16)
+  static constexpr int DH = DH_;          // true head dim
+  static constexpr int DHP = (DH + 15) / 16 * 16;  // Q K^T depth padded to the MMA granule (16)
   static constexpr int BN = BN_;          // keys per K/V tile
   static constexpr int NQ = NQ_;          // 128-row query tiles per CTA
   static constexpr int STAGES = STAGES_;  // K/V ring depth
-  static constexpr int NCH = (DHP + 63) / 64;  // 64-element (128-byte) swizzle chunks along dh
+  static constexpr bool P_SEP = P_SEP_;
+  static constexpr bool L_IN_V = L_IN_V_;
+  static constexpr int NPV = L_IN_V ? (DH + 1 + 15) / 16 * 16 : DHP;  // N of O += P V (O, then l)
+  static constexpr int NCH = (DHP + 63) / 64;    // 64-element (128-byte) swizzle chunks of Q and K
+  static constexpr int NCHV = (NPV + 63) / 64;   // chunks of a V tile (the ones column included)
   static constexpr int Q_TILE_BYTES = NCH * BM * 128;
-  static constexpr int KV_TILE_BYTES = NCH * BN * 128;
+  static constexpr int K_TILE_BYTES = NCH * BN * 128;
+  static constexpr int V_TILE_BYTES = NCHV * BN * 128;
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + NQ * Q_TILE_BYTES;
-  static constexpr int V_OFF = K_OFF + STAGES * KV_TILE_BYTES;
-  static constexpr int BAR_OFF = V_OFF + STAGES * KV_TILE_BYTES;
-  // q_full, k_full[S], v_full[S], kv_empty[S], s_full[NQ], p_full[NQ], o_done[NQ], final
-  static constexpr int NBARS = 1 + 3 * STAGES + 3 * NQ + 1;
+  static constexpr int V_OFF = K_OFF + STAGES * K_TILE_BYTES;
+  static constexpr int BAR_OFF = V_OFF + STAGES * V_TILE_BYTES;
+  // q_full, k_full[S], v_full[S], v_ready[S], kv_empty[S], s_full[NQ], s_free[NQ], p_full[NQ], o_done[NQ],
+  // fin[NQ], and the exp tokens tok[2][4] of the two tiles' warps on each SM sub-partition
+  static constexpr int NBARS = 1 + 4 * STAGES + 5 * NQ + 8;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
-  static constexpr int TM_TILE = 256;                      // TMEM columns per query tile: S | O
+  // TMEM columns of one query tile: S | P (if separate) | O (NPV columns, l at column DH)
+  static constexpr int TM_S = 0;
+  static constexpr int TM_P = P_SEP ? BN : 0;
+  static constexpr int TM_O = BN + (P_SEP ? BN / 2 : 0);
+  static constexpr int TM_USED = TM_O + NPV;
+  static constexpr int TM_TILE = TM_USED <= 256 ? 256 : 512;
   static constexpr int TM_COLS = NQ * TM_TILE;
-  static constexpr int NUM_WARPS = 2 + 4 * NQ;  // producer, MMA issuer, 4 softmax warps per tile
+  // warp 0: TMA producer; warp 1: MMA issuer of tile 0 (and TMEM owner); warps 2 .. 1+4*NQ: softmax
+  // (four per tile); then the V fix-up warp (L_IN_V) and the MMA issuers of tiles 1 .. NQ-1.
+  static constexpr int FIX_WARP = 2 + 4 * NQ;
+  static constexpr int MMA_WARP_T1 = FIX_WARP + (L_IN_V ? 1 : 0);
+  static constexpr int NUM_WARPS = MMA_WARP_T1 + NQ - 1;
   static constexpr int THREADS = 32 * NUM_WARPS;
-  static_assert(DHP % 16 == 0 && DHP <= 256, "MMA N must be a multiple of 16");
-  static_assert(BN % 32 == 0 && BN + DHP <= TM_TILE, "S and O must fit the tile's TMEM columns");
-  static_assert(TM_COLS == 256 || TM_COLS == 512, "TMEM allocation is a power of two");
+  // Of every 8 column pairs, this many take the FMA-pipe exp2 instead of the special-function unit.
+  static constexpr int POLY_PAIRS = SD_POLY_PAIRS >= 0 ? SD_POLY_PAIRS : POLY_;
+  static_assert(NPV % 16 == 0 && NPV <= 256, "MMA N must be a multiple of 16 and at most 256");
+  static_assert(BN % 32 == 0, "S is read in 32-column chunks");
+  static_assert(TM_COLS <= 512, "tensor memory holds 512 columns");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -73,11 +127,14 @@ struct Bars {
   __device__ uint32_t q_full() const { return base; }
   __device__ uint32_t k_full(int s) const { return base + 8 * (1 + s); }
   __device__ uint32_t v_full(int s) const { return base + 8 * (1 + stages + s); }
-  __device__ uint32_t kv_empty(int s) const { return base + 8 * (1 + 2 * stages + s); }
-  __device__ uint32_t s_full(int t) const { return base + 8 * (1 + 3 * stages + t); }
-  __device__ uint32_t p_full(int t) const { return base + 8 * (1 + 3 * stages + nq + t); }
-  __device__ uint32_t o_done(int t) const { return base + 8 * (1 + 3 * stages + 2 * nq + t); }
-  __device__ uint32_t fin() const { return base + 8 * (1 + 3 * stages + 3 * nq); }
+  __device__ uint32_t v_ready(int s) const { return base + 8 * (1 + 2 * stages + s); }
+  __device__ uint32_t kv_empty(int s) const { return base + 8 * (1 + 3 * stages + s); }
+  __device__ uint32_t s_full(int t) const { return base + 8 * (1 + 4 * stages + t); }
+  __device__ uint32_t s_free(int t) const { return base + 8 * (1 + 4 * stages + nq + t); }
+  __device__ uint32_t p_full(int t) const { return base + 8 * (1 + 4 * stages + 2 * nq + t); }
+  __device__ uint32_t o_done(int t) const { return base + 8 * (1 + 4 * stages + 3 * nq + t); }
+  __device__ uint32_t fin() const { return base + 8 * (1 + 4 * stages + 4 * nq); }
+  __device__ uint32_t tok(int t, int q) const { return base + 8 * (1 + 4 * stages + 5 * nq + 4 * t + q); }
 };
 
 // Bounded wait. Returns false if this CTA has aborted or the limit expired (then it raises the
@@ -104,7 +161,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out, int Lq, int Lk,
                    int dh, float scale_log2, unsigned int* err, int debug_flags) {
-  constexpr int BN = C::BN, NQ = C::NQ, STAGES = C::STAGES, NCH = C::NCH, DHP = C::DHP;
+  constexpr int BN = C::BN, NQ = C::NQ, STAGES = C::STAGES, NCH = C::NCH, NCHV = C::NCHV, DHP = C::DHP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -122,14 +179,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bars.k_full(s), 1);
       mbar_init(bars.v_full(s), 1);
-      mbar_init(bars.kv_empty(s), 1);
+      mbar_init(bars.v_ready(s), 1);
+      mbar_init(bars.kv_empty(s), NQ);  // one tcgen05.commit per query tile's MMA issuer
     }
     for (int t = 0; t < NQ; ++t) {
       mbar_init(bars.s_full(t), 1);
+      mbar_init(bars.s_free(t), 128);
       mbar_init(bars.p_full(t), 128);
       mbar_init(bars.o_done(t), 1);
     }
-    mbar_init(bars.fin(), 1);
+    for (int t = 0; t < NQ; ++t) mbar_init(bars.fin() + 8 * t, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bars.tok(i >> 2, i & 3), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -161,15 +221,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int j = 0; j < nkv; ++j) {
         const int s = j % STAGES, round = j / STAGES;
         if (j >= STAGES && !wait_bar(bars.kv_empty(s), (round - 1) & 1, abort_flag, err)) break;
-        mbar_arrive_expect_tx(bars.k_full(s), C::KV_TILE_BYTES);
+        mbar_arrive_expect_tx(bars.k_full(s), C::K_TILE_BYTES);
         for (int c = 0; c < NCH; ++c)
-          tma_load_3d(sbase + C::K_OFF + s * C::KV_TILE_BYTES + c * BN * 128, &tm_k, bars.k_full(s), c * 64,
+          tma_load_3d(sbase + C::K_OFF + s * C::K_TILE_BYTES + c * BN * 128, &tm_k, bars.k_full(s), c * 64,
                       j * BN, bh);
         issued[s] = round + 1;
         if ((debug_flags & 1) && j == 0) break;  // test hook: V tile 0 never arrives
-        mbar_arrive_expect_tx(bars.v_full(s), C::KV_TILE_BYTES);
-        for (int c = 0; c < NCH; ++c)
-          tma_load_3d(sbase + C::V_OFF + s * C::KV_TILE_BYTES + c * BN * 128, &tm_v, bars.v_full(s), c * 64,
+        mbar_arrive_expect_tx(bars.v_full(s), C::V_TILE_BYTES);
+        for (int c = 0; c < NCHV; ++c)
+          tma_load_3d(sbase + C::V_OFF + s * C::V_TILE_BYTES + c * BN * 128, &tm_v, bars.v_full(s), c * 64,
                       j * BN, bh);
       }
       // Drain: every copy this thread issued has landed before the CTA may exit.
@@ -180,83 +240,108 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           if (!(debug_flags & 1)) wait_bar(bars.v_full(s), (issued[s] - 1) & 1, abort_flag, err, false);
         }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp >= C::MMA_WARP_T1) {
+    // ------------------------------------------------------------------ MMA issuer of one tile
+    // One issuing warp per query tile: a tcgen05.mma occupies its issuing thread for tens to
+    // hundreds of cycles, so two tiles' instruction streams must not queue behind each other.
+    const int t = warp == 1 ? 0 : 1 + warp - C::MMA_WARP_T1;
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, DHP, true);
-      auto issue_qk = [&](int t, int s) {
-        const uint32_t d = tmem + t * C::TM_TILE;  // S: columns [0, BN)
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, C::NPV, true);
+      const uint32_t tq = sbase + C::Q_OFF + t * C::Q_TILE_BYTES;
+      auto issue_qk = [&](int s) {  // S = Q K_s^T over the padded head dim
+        const uint32_t d = tmem + t * C::TM_TILE + C::TM_S;
 #pragma unroll
         for (int ks = 0; ks < DHP / 16; ++ks) {
           const uint32_t off = (ks >> 2) * (BM * 128) + (ks & 3) * 32;
           const uint32_t offk = (ks >> 2) * (BN * 128) + (ks & 3) * 32;
-          const uint64_t a = smem_desc(sbase + C::Q_OFF + t * C::Q_TILE_BYTES + off, 16, 1024);
-          const uint64_t b = smem_desc(sbase + C::K_OFF + s * C::KV_TILE_BYTES + offk, 16, 1024);
+          const uint64_t a = smem_desc(tq + off, 16, 1024);
+          const uint64_t b = smem_desc(sbase + C::K_OFF + s * C::K_TILE_BYTES + offk, 16, 1024);
           mma_ss(d, a, b, idesc_qk, ks > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int s, bool first) {
-        const uint32_t d = tmem + t * C::TM_TILE + BN;  // O: columns [BN, BN + DHP)
-        const uint32_t a = tmem + t * C::TM_TILE;       // P: bf16 pairs over S columns [0, BN/2)
+      auto issue_pv = [&](int s, bool first) {  // O (+)= P V_s, P from TMEM (16 keys = 8 columns)
+        const uint32_t d = tmem + t * C::TM_TILE + C::TM_O;
+        const uint32_t a = tmem + t * C::TM_TILE + C::TM_P;
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks) {
-          const uint64_t b = smem_desc(sbase + C::V_OFF + s * C::KV_TILE_BYTES + ks * 16 * 128, BN * 128, 1024);
+          const uint64_t b = smem_desc(sbase + C::V_OFF + s * C::V_TILE_BYTES + ks * 16 * 128, BN * 128, 1024);
           mma_ts(d, a + ks * 8, b, idesc_pv, (!first || ks > 0) ? 1u : 0u);
         }
       };
-      bool ok = wait_bar(bars.q_full(), 0, abort_flag, err) && wait_bar(bars.k_full(0), 0, abort_flag, err);
-      if (ok) {
-        tc_fence_after();
-        for (int t = 0; t < NQ; ++t) {
-          issue_qk(t, 0);
-          mma_commit(bars.s_full(t));
+      bool ok = wait_bar(bars.q_full(), 0, abort_flag, err);
+      // Two pending items per tile, issued in whichever order they become ready: S_jq = Q K_jq^T
+      // (needs K_jq, and the softmax's release of S_{jq-1} -- with P over S, the completion of
+      // P_{jq-1} V), and O += P_jp V_jp (needs P_jp and V_jp). P V goes first when both are
+      // ready: it frees the K/V stage the producer is waiting for.
+      int jq = 0, jp = 0;
+      long long t_idle = clock64();
+      uint32_t spins = 0;
+      while (ok && jp < nkv) {
+#ifdef SD_TRACE
+        if (jp < jq && mbar_test_wait(bars.p_full(t), jp & 1)) {
+          const int cta_ = blockIdx.x + gridDim.x * blockIdx.y;
+          if (cta_ < kTraceCtas && jp < kTraceIters && g_trace[cta_][warp][jp][2] == 0) g_trace[cta_][warp][jp][2] = clock64();
         }
-      }
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int s = j % STAGES;
-        const uint32_t ph = (j / STAGES) & 1;
-        for (int t = 0; ok && t < NQ; ++t) {
-          ok = wait_bar(bars.p_full(t), j & 1, abort_flag, err) &&
-               (t > 0 || wait_bar(bars.v_full(s), ph, abort_flag, err));
-          if (!ok) break;
+#endif
+        const bool can_pv = jp < jq && mbar_test_wait(bars.p_full(t), jp & 1) &&
+                            mbar_test_wait(C::L_IN_V ? bars.v_ready(jp % STAGES) : bars.v_full(jp % STAGES),
+                                           (jp / STAGES) & 1);
+        if (can_pv) {
           tc_fence_after();
-          issue_pv(t, s, j == 0);
+          issue_pv(jp % STAGES, jp == 0);
           mma_commit(bars.o_done(t));
-          if (t == NQ - 1) mma_commit(bars.kv_empty(s));
-          if (j + 1 < nkv) {
-            const int s1 = (j + 1) % STAGES;
-            const uint32_t ph1 = ((j + 1) / STAGES) & 1;
-            // P aliases S: the next S may only be written once this P V has been consumed.
-            ok = wait_bar(bars.o_done(t), j & 1, abort_flag, err) &&
-                 (t > 0 || wait_bar(bars.k_full(s1), ph1, abort_flag, err));
-            if (!ok) break;
-            tc_fence_after();
-            issue_qk(t, s1);
-            mma_commit(bars.s_full(t));
+          mma_commit(bars.kv_empty(jp % STAGES));
+          SD_TR(warp, jp, 1);
+          ++jp;
+          t_idle = clock64();
+          continue;
+        }
+        const bool can_qk = jq < nkv && mbar_test_wait(bars.k_full(jq % STAGES), (jq / STAGES) & 1) &&
+                            (jq == 0 || mbar_test_wait(C::P_SEP ? bars.s_free(t) : bars.o_done(t), (jq - 1) & 1));
+        if (can_qk) {
+          tc_fence_after();
+          issue_qk(jq % STAGES);
+          mma_commit(bars.s_full(t));
+          SD_TR(warp, jq, 0);
+          ++jq;
+          t_idle = clock64();
+          continue;
+        }
+        if ((++spins & 31u) == 0) {
+          if (*abort_flag) break;
+          if (clock64() - t_idle > kWaitLimitCycles) {
+            *abort_flag = 1;
+            atomicOr(err, sd::kDevErrTimeout);
+            break;
           }
         }
       }
       // Drain: all tensor-core work issued by this thread completes before TMEM is released.
-      mma_commit(bars.fin());
-      wait_bar(bars.fin(), 0, abort_flag, err, false);
+      const uint32_t fin = bars.fin() + 8 * t;
+      mma_commit(fin);
+      wait_bar(fin, 0, abort_flag, err, false);
     }
     __syncwarp();
-  } else {
+  } else if (warp < C::FIX_WARP) {
     // ------------------------------------------------------------------ softmax warps
     const int t = (warp - 2) >> 2;  // query tile of this warpgroup
     const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
-    const uint32_t tS = tmem + t * C::TM_TILE + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t tO = tS + BN;
+    const uint32_t tbase = tmem + t * C::TM_TILE + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t tS = tbase + C::TM_S, tP = tbase + C::TM_P, tO = tbase + C::TM_O;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
+    const bool tr = lane == 0;
+    const int trole = warp;
     for (int j = 0; j < nkv; ++j) {
+      if (tr) SD_TR(trole, j, 0);
       // warp-uniform outcome: the tcgen05 copies below are .sync.aligned
       if (!__all_sync(0xffffffffu, wait_bar(bars.s_full(t), j & 1, abort_flag, err))) {
         ok = false;
         break;
       }
+      if (tr) SD_TR(trole, j, 1);
       tc_fence_after();
       float sv[BN];
 #pragma unroll
@@ -267,67 +352,121 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(r[i]);
       }
       tmem_wait_ld();
+      if (tr) SD_TR(trole, j, 2);
+      if constexpr (C::P_SEP) {  // S is in registers: the next S = Q K^T may overwrite it
+        tc_fence_before();
+        mbar_arrive(bars.s_free(t));
+      }
       const int valid = Lk - j * BN;
       if (valid < BN) {
 #pragma unroll
         for (int i = 0; i < BN; ++i)
           if (i >= valid) sv[i] = -INFINITY;
       }
-      float mx = sv[0];
+      // Row max as 16 independent chains of 3-input max, then a short tree.
+      float pm[16];
 #pragma unroll
-      for (int i = 1; i < BN; ++i) mx = fmaxf(mx, sv[i]);
+      for (int k = 0; k < 16; ++k) pm[k] = sv[k];
+#pragma unroll
+      for (int i = 16; i + 32 <= BN; i += 32)
+#pragma unroll
+        for (int k = 0; k < 16; ++k) pm[k] = max3f(pm[k], sv[i + k], sv[i + 16 + k]);
+      if constexpr ((BN / 16) % 2 == 0) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) pm[k] = fmaxf(pm[k], sv[BN - 16 + k]);
+      }
+      const float mx = fmaxf(max3f(max3f(pm[0], pm[1], pm[2]), max3f(pm[3], pm[4], pm[5]), max3f(pm[6], pm[7], pm[8])),
+                             max3f(max3f(pm[9], pm[10], pm[11]), max3f(pm[12], pm[13], pm[14]), pm[15]));
       const float m_new = fmaxf(m_run, mx * scale_log2);
       // Lazy rescale (always on the first tile). The decision is warp-uniform: the tcgen05 copies
-      // of O below are .sync.aligned, and rescaling a row whose max barely moved is still exact.
-      if (__any_sync(0xffffffffu, m_new > m_run + 8.0f)) {
-        const float alpha = ex2_approx(m_run - m_new);
-        l_run *= alpha;
-        if (j > 0) {
-#pragma unroll
-          for (int c = 0; c < DHP / 16; ++c) {
-            uint32_t r[16];
-            tmem_ld16(tO + c * 16, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st16(tO + c * 16, r);
-          }
+      // of O and l below are .sync.aligned, and rescaling a row whose max barely moved is exact.
+      const bool rescale = __any_sync(0xffffffffu, m_new > m_run + 8.0f);
+      if (tr) SD_TR(trole, j, 3);
+      const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
+      if (rescale) m_run = m_new;
+      // Ping-pong: the special-function unit of a sub-partition serves one tile's exp2 phase at a
+      // time; the other tile's warp on it does its row max, P store and S load meanwhile. Tile 0
+      // goes first; each warp hands the token to its partner (same sub-partition) after its exps.
+      constexpr bool kPing = SD_PINGPONG && NQ == 2;
+      if (kPing && (t == 1 || j > 0)) {
+        if (!__all_sync(0xffffffffu, wait_bar(bars.tok(t, quarter), (t == 1 ? j : j - 1) & 1, abort_flag, err))) {
+          ok = false;
+          break;
         }
-        m_run = m_new;
       }
       const float neg_m = -m_run;
-      float rs = 0.f;
+      uint32_t pk[BN / 2];
+      float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < BN / 2; ++i) {
+        float x0, x1, p0, p1;
+        fma2(x0, x1, sv[2 * i], sv[2 * i + 1], scale_log2, scale_log2, neg_m, neg_m);
+        if ((i & 7) < C::POLY_PAIRS) {
+          exp2_poly2(p0, p1, x0, x1);
+        } else {
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
+        }
+        if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, p0, p1);
+        pk[i] = pack_bf16x2(p0, p1);
+      }
+      if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
+      if (kPing) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
+      }
+      if (tr) SD_TR(trole, j, 4);
+      // P_{j-1} V (and the O it accumulates) must be complete before P_j and O are touched.
+      if (C::P_SEP && j > 0) {
+        if (!__all_sync(0xffffffffu, wait_bar(bars.o_done(t), (j - 1) & 1, abort_flag, err))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      if (tr) SD_TR(trole, j, 5);
+      if (rescale && j > 0) {
+#pragma unroll
+        for (int c = 0; c < C::NPV / 16; ++c) {  // O columns, the row-sum column DH among them
+          const uint32_t addr = tO + c * 16;
+          uint32_t r[16];
+          tmem_ld16(addr, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st16(addr, r);
+        }
+      }
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
-        uint32_t pk[16];
+        uint32_t r[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2_approx(fmaf(sv[c * 32 + 2 * i], scale_log2, neg_m));
-          const float p1 = ex2_approx(fmaf(sv[c * 32 + 2 * i + 1], scale_log2, neg_m));
-          rs += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(tS + c * 16, pk);
+        for (int i = 0; i < 16; ++i) r[i] = pk[c * 16 + i];
+        tmem_st16(tP + c * 16, r);
       }
-      l_run += rs;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bars.p_full(t));
+      if (tr) SD_TR(trole, j, 6);
     }
     if (ok && __all_sync(0xffffffffu, wait_bar(bars.o_done(t), (nkv - 1) & 1, abort_flag, err))) {
       tc_fence_after();
       const int qrow = q0 + t * BM + row;
-      const float inv_l = 1.0f / l_run;
+      float lsum = l_run;
       uint32_t packed[DHP / 2];
+      float ov[C::NPV];
 #pragma unroll
-      for (int c = 0; c < DHP / 16; ++c) {
+      for (int c = 0; c < C::NPV / 16; ++c) {
         uint32_t r[16];
         tmem_ld16(tO + c * 16, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          packed[c * 8 + i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv_l, __uint_as_float(r[2 * i + 1]) * inv_l);
+        for (int i = 0; i < 16; ++i) ov[c * 16 + i] = __uint_as_float(r[i]);
       }
+      if constexpr (C::L_IN_V) lsum = ov[C::DH];
+      const float inv_l = 1.0f / lsum;
+#pragma unroll
+      for (int i = 0; i < DHP / 2; ++i) packed[i] = pack_bf16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l);
       if (qrow < Lq) {
         uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * Lq + qrow) * dh);
         const int n16 = dh / 8;  // 16-byte groups of 8 bf16
@@ -335,6 +474,24 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int i = 0; i < DHP / 8; ++i)
           if (i < n16) dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
       }
+    }
+  }
+
+  if (C::L_IN_V && warp == C::FIX_WARP) {
+    // ------------------------------------------------------------------ V fix-up warp
+    // Writes bf16 1.0 into column DH of every landed V tile (128-byte swizzled rows: the 16-byte
+    // granule g of row r sits at granule g ^ (r % 8)), then hands the tile to the MMA issuer.
+    constexpr int ch = C::DH / 64, byte = (C::DH % 64) * 2, g = byte >> 4, gb = byte & 15;
+    for (int j = 0; j < nkv; ++j) {
+      const int s = j % STAGES;
+      if (!__all_sync(0xffffffffu, wait_bar(bars.v_full(s), (j / STAGES) & 1, abort_flag, err))) break;
+      uint8_t* vt = smem + C::V_OFF + s * C::V_TILE_BYTES + ch * BN * 128;
+#pragma unroll
+      for (int r = lane; r < BN; r += 32)
+        *reinterpret_cast<uint16_t*>(vt + r * 128 + ((g ^ (r & 7)) << 4) + gb) = 0x3F80u;  // bf16 1.0
+      fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.v_ready(s));
     }
   }
 
@@ -390,9 +547,17 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
   unsigned int* err = sd::device_status_word();
   if (!err) return SD_ERR_CUDA;
   auto kern = attn_fwd_sm100<C>;
-  st = sd::cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES),
-                      "cudaFuncSetAttribute(attention smem)");
+  static std::atomic<uint64_t> smem_set{0};  // one bit per device: opt-in to large shared memory done
+  int dev = 0;
+  st = sd::cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
   if (st != SD_OK) return st;
+  const uint64_t bit = uint64_t(1) << (dev & 63);
+  if (!(smem_set.load(std::memory_order_acquire) & bit)) {
+    st = sd::cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES),
+                        "cudaFuncSetAttribute(attention smem)");
+    if (st != SD_OK) return st;
+    smem_set.fetch_or(bit, std::memory_order_acq_rel);
+  }
   const dim3 grid(static_cast<unsigned>((Lq + BM * C::NQ - 1) / (BM * C::NQ)), static_cast<unsigned>(BH));
   const float scale_log2 = scale * 1.4426950408889634f;
   kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), static_cast<int>(Lq),
@@ -422,13 +587,21 @@ extern "C" sd_status sd_attention(const void* q, const void* k, const void* v, v
     return sd::fail(SD_ERR_INVALID_ARG, "sd_attention: o overlaps q, k or v");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (dh) {
-    case 40: return launch<Cfg<48, 128, 2, 3>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
-    case 64: return launch<Cfg<64, 128, 2, 3>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
-    case 80: return launch<Cfg<80, 128, 2, 2>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
-    default: return launch<Cfg<160, 64, 1, 3>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
+    case 40: return launch<Cfg<40, 128, 2, SD_STAGES_SMALL, true, true, 2>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
+    case 64: return launch<Cfg<64, 128, 2, SD_STAGES_SMALL, true, false>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
+    case 80: return launch<Cfg<80, 128, 2, 2, false, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
+    default: return launch<Cfg<160, 64, 1, 3, true, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
   }
 }
 
 // Test hook (declared in sd_kernels.h): bit 0 makes the next attention launches skip their first
 // V tile so that the kernel's bounded wait expires and reports SD_ERR_TIMEOUT.
 extern "C" void sd_debug_set_fault(int flags) { g_debug_flags = flags; }
+
+#ifdef SD_TRACE
+// Tuning builds only: copies the phase timestamps to host memory.
+extern "C" int sd_debug_trace(void* host, int64_t bytes) {
+  if (bytes < static_cast<int64_t>(sizeof(g_trace))) return -1;
+  return cudaMemcpyFromSymbol(host, g_trace, sizeof(g_trace)) == cudaSuccess ? 0 : -2;
+}
+#endif

@@ -72,10 +72,12 @@ __device__ __forceinline__ void st_stream(float4* p, float4 v) {
                : "memory");
 }
 
-// Reduces the thread's triple over the CTA, publishes it to the cluster, and returns (in shared
-// memory) the group's mean and rstd as merged by every CTA in the same order.
+// Reduces the thread's triple over the CTA, pushes the CTA's triple into slot `rank` of every
+// cluster peer's shared memory, and after one cluster barrier merges the slots in rank order, so
+// that every CTA obtains the same mean and rstd (left in shared memory). No CTA touches another's
+// shared memory after the barrier, so CTAs may exit without a second cluster-wide sync.
 __device__ __forceinline__ void cluster_group_stats(Stats st, float eps, float* s_mean, float* s_rstd,
-                                                    Stats* s_warp, Stats* s_cta) {
+                                                    Stats* s_warp, Stats* s_all) {
   cg::cluster_group cluster = cg::this_cluster();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -85,17 +87,18 @@ __device__ __forceinline__ void cluster_group_stats(Stats st, float eps, float* 
   }
   if (lane == 0) s_warp[warp] = st;
   __syncthreads();
+  const unsigned cs = cluster.num_blocks();
   if (threadIdx.x == 0) {
     Stats a = s_warp[0];
 #pragma unroll
     for (int w = 1; w < kWarps; ++w) a = merge(a, s_warp[w]);
-    *s_cta = a;
+    const unsigned rank = cluster.block_rank();
+    for (unsigned r = 0; r < cs; ++r) *cluster.map_shared_rank(&s_all[rank], r) = a;
   }
-  cluster.sync();  // every CTA's triple is now visible to the cluster
+  cluster.sync();  // release/acquire: every peer's slot write is visible
   if (threadIdx.x == 0) {
-    const unsigned cs = cluster.num_blocks();
-    Stats a = *cluster.map_shared_rank(s_cta, 0);
-    for (unsigned r = 1; r < cs; ++r) a = merge(a, *cluster.map_shared_rank(s_cta, r));
+    Stats a = s_all[0];
+    for (unsigned r = 1; r < cs; ++r) a = merge(a, s_all[r]);
     const float var = a.n > 0.f ? fmaxf(a.m2 / a.n, 0.f) : 0.f;
     *s_mean = a.mean;
     *s_rstd = rsqrtf(var + eps);
@@ -111,7 +114,7 @@ __global__ void __launch_bounds__(kThreads) gn_resident(const float* x, const fl
                                                         int group_elems, int chunk, int hw, int cpg, int groups,
                                                         float eps) {
   __shared__ Stats s_warp[kWarps];
-  __shared__ Stats s_cta;
+  __shared__ Stats s_all[kMaxCluster];
   __shared__ float s_mean, s_rstd;
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
@@ -144,7 +147,7 @@ __global__ void __launch_bounds__(kThreads) gn_resident(const float* x, const fl
       st.m2 += a * a + b * b + c * c + d * d;
     }
   }
-  cluster_group_stats(st, eps, &s_mean, &s_rstd, s_warp, &s_cta);
+  cluster_group_stats(st, eps, &s_mean, &s_rstd, s_warp, s_all);
   const float mean = s_mean, rstd = s_rstd;
 
   float4* yg = reinterpret_cast<float4*>(y + base);
@@ -160,7 +163,6 @@ __global__ void __launch_bounds__(kThreads) gn_resident(const float* x, const fl
                                       fmaf(v[i].w, a, b)));
     }
   }
-  cluster.sync();  // peers read s_cta through distributed shared memory; keep it alive until they are done
 }
 
 // Streaming path: any shape and alignment. CTA `rank` of the cluster owns elements [lo, hi) of the
@@ -171,7 +173,7 @@ __global__ void __launch_bounds__(kThreads) gn_streaming(const float* x, const f
                                                          int64_t group_elems, int64_t chunk, int64_t hw, int cpg,
                                                          int groups, float eps) {
   __shared__ Stats s_warp[kWarps];
-  __shared__ Stats s_cta;
+  __shared__ Stats s_all[kMaxCluster];
   __shared__ float s_mean, s_rstd;
   cg::cluster_group cluster = cg::this_cluster();
   const int64_t rank = cluster.block_rank();
@@ -203,14 +205,13 @@ __global__ void __launch_bounds__(kThreads) gn_streaming(const float* x, const f
     }
     st = merge(st, r);
   }
-  cluster_group_stats(st, eps, &s_mean, &s_rstd, s_warp, &s_cta);
+  cluster_group_stats(st, eps, &s_mean, &s_rstd, s_warp, s_all);
   const float mean = s_mean, rstd = s_rstd;
   for (int64_t e = lo + threadIdx.x; e < hi; e += kThreads) {
     const int c = g * cpg + static_cast<int>(e / hw);
     const float a = rstd * __ldg(gamma + c);
     yg[e] = fmaf(xg[e], a, fmaf(-mean, a, __ldg(beta + c)));
   }
-  cluster.sync();
 }
 
 template <int ITEMS>
