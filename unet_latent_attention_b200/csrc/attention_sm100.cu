@@ -107,11 +107,13 @@ struct Cfg {
   static constexpr int TM_USED = TM_O + NPV;
   static constexpr int TM_TILE = TM_USED <= 256 ? 256 : 512;
   static constexpr int TM_COLS = NQ * TM_TILE;
-  // warp 0: TMA producer; warp 1: MMA issuer of tile 0 (and TMEM owner); warps 2 .. 1+4*NQ: softmax
-  // (four per tile); then the V fix-up warp (L_IN_V) and the MMA issuers of tiles 1 .. NQ-1.
-  static constexpr int FIX_WARP = 2 + 4 * NQ;
-  static constexpr int MMA_WARP_T1 = FIX_WARP + (L_IN_V ? 1 : 0);
-  static constexpr int NUM_WARPS = MMA_WARP_T1 + NQ - 1;
+  // Warpgroup 0 holds the helpers -- warp 0: TMA producer; warp 1: MMA issuer of tile 0 (and TMEM
+  // owner); warp 2: MMA issuer of tile 1; warp 3: V fix-up (L_IN_V) -- and warpgroups 1 .. NQ run
+  // the softmax of one query tile each (warp w reads TMEM lane quarter w % 4).
+  static_assert(NQ <= 2, "two MMA issuers in warpgroup 0");
+  static constexpr int FIX_WARP = 3;
+  static constexpr int SOFT_WARP0 = 4;
+  static constexpr int NUM_WARPS = 4 + 4 * NQ;
   static constexpr int THREADS = 32 * NUM_WARPS;
   // Of every 8 column pairs, this many take the FMA-pipe exp2 instead of the special-function unit.
   static constexpr int POLY_PAIRS = SD_POLY_PAIRS >= 0 ? SD_POLY_PAIRS : POLY_;
@@ -207,6 +209,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  if (warp < C::SOFT_WARP0) {
+  // ==================================================================== helper warpgroup
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -240,11 +244,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           if (!(debug_flags & 1)) wait_bar(bars.v_full(s), (issued[s] - 1) & 1, abort_flag, err, false);
         }
     }
-  } else if (warp == 1 || warp >= C::MMA_WARP_T1) {
+  } else if (warp == 1 || (NQ == 2 && warp == 2)) {
     // ------------------------------------------------------------------ MMA issuer of one tile
     // One issuing warp per query tile: a tcgen05.mma occupies its issuing thread for tens to
     // hundreds of cycles, so two tiles' instruction streams must not queue behind each other.
-    const int t = warp == 1 ? 0 : 1 + warp - C::MMA_WARP_T1;
+    const int t = warp - 1;
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, C::NPV, true);
@@ -323,9 +327,35 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       wait_bar(fin, 0, abort_flag, err, false);
     }
     __syncwarp();
-  } else if (warp < C::FIX_WARP) {
+  } else if (C::L_IN_V && warp == C::FIX_WARP) {
+
+    // ------------------------------------------------------------------ V fix-up warp
+    // Writes bf16 1.0 into column DH of every landed V tile (128-byte swizzled rows: the 16-byte
+    // granule g of row r sits at granule g ^ (r % 8)), then hands the tile to the MMA issuer.
+    constexpr int ch = C::DH / 64, byte = (C::DH % 64) * 2, g = byte >> 4, gb = byte & 15;
+    for (int j = 0; j < nkv; ++j) {
+      const int s = j % STAGES;
+      if (!__all_sync(0xffffffffu, wait_bar(bars.v_full(s), (j / STAGES) & 1, abort_flag, err))) break;
+      uint8_t* vt = smem + C::V_OFF + s * C::V_TILE_BYTES + ch * BN * 128;
+#pragma unroll
+      for (int r = lane; r < BN; r += 32)
+        *reinterpret_cast<uint16_t*>(vt + r * 128 + ((g ^ (r & 7)) << 4) + gb) = 0x3F80u;  // bf16 1.0
+      fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.v_ready(s));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TM_COLS);
+  }
+  } else {
+  // ==================================================================== softmax warpgroups
+  {
     // ------------------------------------------------------------------ softmax warps
-    const int t = (warp - 2) >> 2;  // query tile of this warpgroup
+    const int t = (warp - C::SOFT_WARP0) >> 2;  // query tile of this warpgroup
     const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
     const uint32_t tbase = tmem + t * C::TM_TILE + (static_cast<uint32_t>(quarter * 32) << 16);
@@ -398,17 +428,28 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       uint32_t pk[BN / 2];
       float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < BN / 2; ++i) {
-        float x0, x1, p0, p1;
-        fma2(x0, x1, sv[2 * i], sv[2 * i + 1], scale_log2, scale_log2, neg_m, neg_m);
-        if ((i & 7) < C::POLY_PAIRS) {
-          exp2_poly2(p0, p1, x0, x1);
-        } else {
-          p0 = ex2_approx(x0);
-          p1 = ex2_approx(x1);
+      for (int b = 0; b < BN / 32; ++b) {
+        // 16 column pairs at a time: all arguments, then all exponentials, then the packing, so
+        // that many independent special-function operations are in flight per warp.
+        float x[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          fma2(x[2 * i], x[2 * i + 1], sv[32 * b + 2 * i], sv[32 * b + 2 * i + 1], scale_log2, scale_log2, neg_m,
+               neg_m);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if ((i & 7) < C::POLY_PAIRS) {
+            exp2_poly2(x[2 * i], x[2 * i + 1], x[2 * i], x[2 * i + 1]);
+          } else {
+            x[2 * i] = ex2_approx(x[2 * i]);
+            x[2 * i + 1] = ex2_approx(x[2 * i + 1]);
+          }
         }
-        if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, p0, p1);
-        pk[i] = pack_bf16x2(p0, p1);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x[2 * i], x[2 * i + 1]);
+          pk[16 * b + i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+        }
       }
       if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
       if (kPing) {
@@ -476,30 +517,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
     }
   }
-
-  if (C::L_IN_V && warp == C::FIX_WARP) {
-    // ------------------------------------------------------------------ V fix-up warp
-    // Writes bf16 1.0 into column DH of every landed V tile (128-byte swizzled rows: the 16-byte
-    // granule g of row r sits at granule g ^ (r % 8)), then hands the tile to the MMA issuer.
-    constexpr int ch = C::DH / 64, byte = (C::DH % 64) * 2, g = byte >> 4, gb = byte & 15;
-    for (int j = 0; j < nkv; ++j) {
-      const int s = j % STAGES;
-      if (!__all_sync(0xffffffffu, wait_bar(bars.v_full(s), (j / STAGES) & 1, abort_flag, err))) break;
-      uint8_t* vt = smem + C::V_OFF + s * C::V_TILE_BYTES + ch * BN * 128;
-#pragma unroll
-      for (int r = lane; r < BN; r += 32)
-        *reinterpret_cast<uint16_t*>(vt + r * 128 + ((g ^ (r & 7)) << 4) + gb) = 0x3F80u;  // bf16 1.0
-      fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bars.v_ready(s));
-    }
-  }
-
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::TM_COLS);
   }
 }
 
@@ -586,8 +605,16 @@ extern "C" sd_status sd_attention(const void* q, const void* k, const void* v, v
   if (sd::overlaps(o, qbytes, q, qbytes) || sd::overlaps(o, qbytes, k, kvbytes) || sd::overlaps(o, qbytes, v, kvbytes))
     return sd::fail(SD_ERR_INVALID_ARG, "sd_attention: o overlaps q, k or v");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (Lk <= 96) {  // short key sequence (the 77-token text context): one 96-key tile, no online rescale
+    switch (dh) {
+      case 40: return launch<Cfg<40, 96, 2, 2, true, true, 0>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
+      case 64: return launch<Cfg<64, 96, 2, 2, true, false>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
+      case 80: return launch<Cfg<80, 96, 2, 2, true, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
+      default: break;  // dh = 160 already uses 64-key tiles
+    }
+  }
   switch (dh) {
-    case 40: return launch<Cfg<40, 128, 2, SD_STAGES_SMALL, true, true, 2>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
+    case 40: return launch<Cfg<40, 128, 2, SD_STAGES_SMALL, true, true, 0>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
     case 64: return launch<Cfg<64, 128, 2, SD_STAGES_SMALL, true, false>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
     case 80: return launch<Cfg<80, 128, 2, 2, false, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
     default: return launch<Cfg<160, 64, 1, 3, true, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);

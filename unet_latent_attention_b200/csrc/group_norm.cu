@@ -28,11 +28,14 @@ namespace cg = cooperative_groups;
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kWarps = kThreads / 32;
+constexpr int kThreads = 256;  // streaming path
+constexpr int kMaxWarps = 32;
 constexpr int kMaxCluster = 8;
 constexpr int kMaxItems = 16;  // float4 per thread on the resident path
-constexpr int64_t kResidentCap = static_cast<int64_t>(kThreads) * 4 * kMaxItems;  // elements per CTA
+
+#ifndef SD_GN_POLICY
+#define SD_GN_POLICY 0
+#endif
 
 struct Stats {
   float n, mean, m2;
@@ -90,8 +93,8 @@ __device__ __forceinline__ void cluster_group_stats(Stats st, float eps, float* 
   const unsigned cs = cluster.num_blocks();
   if (threadIdx.x == 0) {
     Stats a = s_warp[0];
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) a = merge(a, s_warp[w]);
+    const int nw = blockDim.x >> 5;
+    for (int w = 1; w < nw; ++w) a = merge(a, s_warp[w]);
     const unsigned rank = cluster.block_rank();
     for (unsigned r = 0; r < cs; ++r) *cluster.map_shared_rank(&s_all[rank], r) = a;
   }
@@ -108,12 +111,12 @@ __device__ __forceinline__ void cluster_group_stats(Stats st, float eps, float* 
 
 // Resident path: one cluster of `cs` CTAs per (b, g); CTA `rank` owns elements
 // [rank*chunk, (rank+1)*chunk) of the group, chunk a multiple of 4, held in registers.
-template <int ITEMS>
-__global__ void __launch_bounds__(kThreads) gn_resident(const float* x, const float* __restrict__ gamma,
+template <int ITEMS, int THREADS>
+__global__ void __launch_bounds__(THREADS) gn_resident(const float* x, const float* __restrict__ gamma,
                                                         const float* __restrict__ beta, float* y,
                                                         int group_elems, int chunk, int hw, int cpg, int groups,
                                                         float eps) {
-  __shared__ Stats s_warp[kWarps];
+  __shared__ Stats s_warp[THREADS / 32];
   __shared__ Stats s_all[kMaxCluster];
   __shared__ float s_mean, s_rstd;
   cg::cluster_group cluster = cg::this_cluster();
@@ -127,14 +130,14 @@ __global__ void __launch_bounds__(kThreads) gn_resident(const float* x, const fl
   float4 v[ITEMS];
 #pragma unroll
   for (int i = 0; i < ITEMS; ++i) {
-    const int idx = threadIdx.x + i * kThreads;
+    const int idx = threadIdx.x + i * THREADS;
     v[i] = idx < n4 ? ld_stream(xg + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   // Thread triple: exact mean of its values, then M2 about it.
   float sum = 0.f, cnt = 0.f;
 #pragma unroll
   for (int i = 0; i < ITEMS; ++i) {
-    if (threadIdx.x + i * kThreads < n4) {
+    if (threadIdx.x + i * THREADS < n4) {
       sum += (v[i].x + v[i].y) + (v[i].z + v[i].w);
       cnt += 4.f;
     }
@@ -142,7 +145,7 @@ __global__ void __launch_bounds__(kThreads) gn_resident(const float* x, const fl
   Stats st{cnt, cnt > 0.f ? sum / cnt : 0.f, 0.f};
 #pragma unroll
   for (int i = 0; i < ITEMS; ++i) {
-    if (threadIdx.x + i * kThreads < n4) {
+    if (threadIdx.x + i * THREADS < n4) {
       const float a = v[i].x - st.mean, b = v[i].y - st.mean, c = v[i].z - st.mean, d = v[i].w - st.mean;
       st.m2 += a * a + b * b + c * c + d * d;
     }
@@ -154,7 +157,7 @@ __global__ void __launch_bounds__(kThreads) gn_resident(const float* x, const fl
   const int e0 = rank * chunk;
 #pragma unroll
   for (int i = 0; i < ITEMS; ++i) {
-    const int idx = threadIdx.x + i * kThreads;
+    const int idx = threadIdx.x + i * THREADS;
     if (idx < n4) {
       const int c = g * cpg + (e0 + idx * 4) / hw;  // hw % 4 == 0: a float4 never straddles channels
       const float a = rstd * __ldg(gamma + c);
@@ -172,7 +175,7 @@ __global__ void __launch_bounds__(kThreads) gn_streaming(const float* x, const f
                                                          const float* __restrict__ beta, float* y,
                                                          int64_t group_elems, int64_t chunk, int64_t hw, int cpg,
                                                          int groups, float eps) {
-  __shared__ Stats s_warp[kWarps];
+  __shared__ Stats s_warp[kThreads / 32];
   __shared__ Stats s_all[kMaxCluster];
   __shared__ float s_mean, s_rstd;
   cg::cluster_group cluster = cg::this_cluster();
@@ -214,13 +217,13 @@ __global__ void __launch_bounds__(kThreads) gn_streaming(const float* x, const f
   }
 }
 
-template <int ITEMS>
+template <int ITEMS, int THREADS>
 cudaError_t launch_resident(dim3 grid, int cs, cudaStream_t s, const float* x, const float* gamma,
                             const float* beta, float* y, int group_elems, int chunk, int hw, int cpg, int groups,
                             float eps) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(THREADS);
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -229,7 +232,7 @@ cudaError_t launch_resident(dim3 grid, int cs, cudaStream_t s, const float* x, c
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, gn_resident<ITEMS>, x, gamma, beta, y, group_elems, chunk, hw, cpg, groups, eps);
+  return cudaLaunchKernelEx(&cfg, gn_resident<ITEMS, THREADS>, x, gamma, beta, y, group_elems, chunk, hw, cpg, groups, eps);
 }
 
 }  // namespace
@@ -255,29 +258,44 @@ extern "C" sd_status sd_group_norm(const float* x, const float* gamma, const flo
     return sd::fail(SD_ERR_INVALID_ARG, "sd_group_norm: y overlaps an input (only y == x is allowed)");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
-  // Resident path: the smallest cluster (power of two <= 8) that holds the group in registers and
-  // gives at least two CTAs per SM; chunk must be a multiple of 4 elements.
+  // Resident path: a (cluster size, CTA size) pair that holds the group in registers (at most
+  // kMaxItems float4 per thread, 8 for 1024-thread CTAs) with chunk a multiple of 4 elements.
+  // Policy (measured on the SD shapes): the smallest cluster and CTA size that still put about
+  // one CTA on every SM.
   const bool vec_ok = hw % 4 == 0 && sd::aligned16(x) && sd::aligned16(y);
-  int cs = 0;
+  int cs = 0, threads = 0;
   if (vec_ok) {
-    const int64_t want_ctas = 2 * static_cast<int64_t>(sd::sm_count());
-    for (int c = 1; c <= kMaxCluster; c *= 2) {
-      if (group_elems % (4 * c) != 0 || group_elems / c > kResidentCap) continue;
-      cs = c;
-      if (n_groups * c >= want_ctas) break;
+    const int64_t sms = sd::sm_count();
+    const int64_t want = SD_GN_POLICY == 0 ? 2 * sms : SD_GN_POLICY == 1 ? 0 : sms;
+    const int tlist0[3] = {256, 512, 1024};
+    const int tlist1[3] = {1024, 512, 256};
+    const int* tl = SD_GN_POLICY == 0 ? tlist0 : tlist1;
+    for (int ti = 0; ti < 3 && !cs; ++ti) {
+      const int th = tl[ti];
+      const int max_items = th == 1024 ? 8 : kMaxItems;
+      for (int c = 1; c <= kMaxCluster; c *= 2) {
+        if (group_elems % (4 * c) != 0 || group_elems / c > int64_t(th) * 4 * max_items) continue;
+        if (n_groups * c < want && c < kMaxCluster) continue;
+        cs = c;
+        threads = th;
+        break;
+      }
     }
   }
   cudaError_t err;
   if (cs > 0) {
     const int chunk = static_cast<int>(group_elems / cs);
-    const int need = (chunk / 4 + kThreads - 1) / kThreads;
+    const int need = (chunk / 4 + threads - 1) / threads;
     const dim3 grid(static_cast<unsigned>(n_groups * cs));
     const int ge = static_cast<int>(group_elems), ihw = static_cast<int>(hw), icpg = static_cast<int>(cpg),
               ig = static_cast<int>(groups);
-#define SD_GN_CASE(N) \
-  if (need <= N) err = launch_resident<N>(grid, cs, s, x, gamma, beta, y, ge, chunk, ihw, icpg, ig, eps); else
-    SD_GN_CASE(1) SD_GN_CASE(2) SD_GN_CASE(3) SD_GN_CASE(4) SD_GN_CASE(5) SD_GN_CASE(6) SD_GN_CASE(8)
-    SD_GN_CASE(10) SD_GN_CASE(12) SD_GN_CASE(16) err = cudaErrorInvalidValue;
+#define SD_GN_CASE(N, T) \
+  if (threads == T && need <= N) err = launch_resident<N, T>(grid, cs, s, x, gamma, beta, y, ge, chunk, ihw, icpg, ig, eps); else
+#define SD_GN_T(T) SD_GN_CASE(1, T) SD_GN_CASE(2, T) SD_GN_CASE(3, T) SD_GN_CASE(4, T) SD_GN_CASE(5, T) \
+    SD_GN_CASE(6, T) SD_GN_CASE(8, T)
+    SD_GN_T(256) SD_GN_T(512) SD_GN_T(1024) SD_GN_CASE(10, 256) SD_GN_CASE(12, 256) SD_GN_CASE(16, 256)
+    SD_GN_CASE(10, 512) SD_GN_CASE(12, 512) SD_GN_CASE(16, 512) err = cudaErrorInvalidValue;
+#undef SD_GN_T
 #undef SD_GN_CASE
   } else {
     // Streaming path: a cluster of up to 8 CTAs per group, each with at least 1024 elements.
