@@ -42,7 +42,7 @@ def test_attention_argument_errors(L):
     assert L.sd_attention(P, P, P, P + 64, 1, 1, 8, 8, 40, 1.0, None) == 1 and "overlap" in _err(L)
     assert L.sd_attention(0, 0, 0, 0, 0, 8, 8, 8, 40, 1.0, None) == 0  # empty: no launch
     assert L.sd_attention(0, 0, 0, 0, 1, 1, 4, 0, 40, 1.0, None) == 1  # Lq >= 1 needs a key
-    assert L.sd_attention(P, P, P, P, 70000, 1, 8, 8, 40, 1.0, None) == 2
+    assert L.sd_attention(P, P, P, P, 1 << 31, 1, 8, 8, 40, 1.0, None) == 2
 
 
 def test_group_norm_argument_errors(L):

@@ -99,3 +99,24 @@ def test_workload_shapes(cuda, wid, label, shape):
         rows = _sampled_rows(shape, 96, wid)
         ref = oracle.attention_rows(q, k, v, rows)
         _check(o[rows[:, 0], rows[:, 1], rows[:, 2]], ref)
+
+
+@pytest.mark.parametrize("dh,heads,Lq,Lk", [(40, 80, 256, 640), (64, 80, 256, 1000), (80, 80, 256, 700),
+                                            (160, 120, 128, 300), (40, 96, 300, 129)])
+def test_split_items_persistent_schedule(cuda, dh, heads, Lq, Lk):
+    # more query-tile items than SMs: the persistent grid splits items between neighbouring CTAs
+    # and merges the two partial results; compared in full with the oracle
+    q, k, v = _qkv(2, heads, Lq, Lk, dh, 9000 + dh + Lk)
+    o = _run(q, k, v, cuda)
+    _check(o, oracle.attention(q, k, v))
+
+
+def test_repeated_launches_reuse_the_hand_off_flags(cuda):
+    # the split hand-off flags must return to zero after every launch (graph replays rely on it)
+    q, k, v = _qkv(2, 80, 256, 640, 40, 9100)
+    ref = oracle.attention(q, k, v)
+    qd, kd, vd = q.to(cuda), k.to(cuda), v.to(cuda)
+    for _ in range(3):
+        o = sdk.sd_attention(qd, kd, vd)
+        sdk.sd_device_status()
+        _check(o.float().cpu().numpy(), ref)

@@ -32,6 +32,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <algorithm>
 #include <cmath>
 #include <mutex>
 
@@ -65,8 +66,12 @@ __device__ long long g_trace[kTraceCtas][12][kTraceIters][kTraceSlots];
 #define SD_PINGPONG 1  // alternate the two query tiles' exp2 phases on each SM sub-partition
 #endif
 
+#ifndef SD_MMA_IDLE_NS
+#define SD_MMA_IDLE_NS 0  // backoff of the MMA issuers' idle poll, in ns (0 = spin)
+#endif
+
 #ifndef SD_STAGES_SMALL
-#define SD_STAGES_SMALL 5  // K/V ring depth for head dims <= 64 (one 16 KB K and V tile per stage)
+#define SD_STAGES_SMALL 4  // K/V ring depth for head dims <= 64 (one 16 KB K and V tile per stage)
 #endif
 
 constexpr int BM = 128;                               // query rows per tile = TMEM lanes
@@ -92,12 +97,14 @@ struct Cfg {
   static constexpr int K_TILE_BYTES = NCH * BN * 128;
   static constexpr int V_TILE_BYTES = NCHV * BN * 128;
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + NQ * Q_TILE_BYTES;
+  // Two Q buffers (when shared memory allows) let the next item's Q load during this one.
+  static constexpr int QBUF = 2 * NQ * NCH * BM * 128 + STAGES * (NCH + NCHV) * BN * 128 <= 200 * 1024 ? 2 : 1;
+  static constexpr int K_OFF = Q_OFF + QBUF * NQ * Q_TILE_BYTES;
   static constexpr int V_OFF = K_OFF + STAGES * K_TILE_BYTES;
   static constexpr int BAR_OFF = V_OFF + STAGES * V_TILE_BYTES;
   // q_full, k_full[S], v_full[S], v_ready[S], kv_empty[S], s_full[NQ], s_free[NQ], p_full[NQ], o_done[NQ],
-  // fin[NQ], and the exp tokens tok[2][4] of the two tiles' warps on each SM sub-partition
-  static constexpr int NBARS = 1 + 4 * STAGES + 5 * NQ + 8;
+  // fin[NQ], the exp tokens tok[2][4] of the two tiles' warps on each SM sub-partition, q_empty
+  static constexpr int NBARS = 2 + 4 * STAGES + 5 * NQ + 8 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
   // TMEM columns of one query tile: S | P (if separate) | O (NPV columns, l at column DH)
@@ -115,6 +122,8 @@ struct Cfg {
   static constexpr int SOFT_WARP0 = 4;
   static constexpr int NUM_WARPS = 4 + 4 * NQ;
   static constexpr int THREADS = 32 * NUM_WARPS;
+  // Split-item hand-off slot: raw O (NPV fp32 per row) and (m, l) per row of the NQ tiles.
+  static constexpr int SLOT_FLOATS = NQ * BM * (NPV + 2);
   // Of every 8 column pairs, this many take the FMA-pipe exp2 instead of the special-function unit.
   static constexpr int POLY_PAIRS = SD_POLY_PAIRS >= 0 ? SD_POLY_PAIRS : POLY_;
   static_assert(NPV % 16 == 0 && NPV <= 256, "MMA N must be a multiple of 16 and at most 256");
@@ -126,17 +135,18 @@ struct Cfg {
 struct Bars {
   uint32_t base;
   int stages, nq;
-  __device__ uint32_t q_full() const { return base; }
-  __device__ uint32_t k_full(int s) const { return base + 8 * (1 + s); }
-  __device__ uint32_t v_full(int s) const { return base + 8 * (1 + stages + s); }
-  __device__ uint32_t v_ready(int s) const { return base + 8 * (1 + 2 * stages + s); }
-  __device__ uint32_t kv_empty(int s) const { return base + 8 * (1 + 3 * stages + s); }
-  __device__ uint32_t s_full(int t) const { return base + 8 * (1 + 4 * stages + t); }
-  __device__ uint32_t s_free(int t) const { return base + 8 * (1 + 4 * stages + nq + t); }
-  __device__ uint32_t p_full(int t) const { return base + 8 * (1 + 4 * stages + 2 * nq + t); }
-  __device__ uint32_t o_done(int t) const { return base + 8 * (1 + 4 * stages + 3 * nq + t); }
-  __device__ uint32_t fin() const { return base + 8 * (1 + 4 * stages + 4 * nq); }
-  __device__ uint32_t tok(int t, int q) const { return base + 8 * (1 + 4 * stages + 5 * nq + 4 * t + q); }
+  __device__ uint32_t q_full(int b) const { return base + 8 * b; }
+  __device__ uint32_t k_full(int s) const { return base + 8 * (2 + s); }
+  __device__ uint32_t v_full(int s) const { return base + 8 * (2 + stages + s); }
+  __device__ uint32_t v_ready(int s) const { return base + 8 * (2 + 2 * stages + s); }
+  __device__ uint32_t kv_empty(int s) const { return base + 8 * (2 + 3 * stages + s); }
+  __device__ uint32_t s_full(int t) const { return base + 8 * (2 + 4 * stages + t); }
+  __device__ uint32_t s_free(int t) const { return base + 8 * (2 + 4 * stages + nq + t); }
+  __device__ uint32_t p_full(int t) const { return base + 8 * (2 + 4 * stages + 2 * nq + t); }
+  __device__ uint32_t o_done(int t) const { return base + 8 * (2 + 4 * stages + 3 * nq + t); }
+  __device__ uint32_t fin() const { return base + 8 * (2 + 4 * stages + 4 * nq); }
+  __device__ uint32_t tok(int t, int q) const { return base + 8 * (2 + 4 * stages + 5 * nq + 4 * t + q); }
+  __device__ uint32_t q_empty(int b) const { return base + 8 * (2 + 4 * stages + 5 * nq + 8 + b); }
 };
 
 // Bounded wait. Returns false if this CTA has aborted or the limit expired (then it raises the
@@ -158,11 +168,30 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile in
   }
 }
 
+// Persistent schedule: the work is items x nkv units (an item = NQ query tiles of one (b, h); a
+// unit = one K/V tile of it). CTA c owns units [c U / G, (c+1) U / G) in item-major order, so every
+// CTA gets the same amount of work whatever the number of SMs; with G <= items each range spans at
+// least nkv units, so an item is split across at most two CTAs: a "head" piece [0, k) at the end
+// of CTA c's range and a "tail" piece [k, nkv) at the start of CTA c+1's range.
+struct Seg {
+  int it, kb, ke;
+};
+__device__ __forceinline__ bool next_seg(long long& u, long long u1, int nkv, Seg& sg) {
+  if (u >= u1) return false;
+  sg.it = static_cast<int>(u / nkv);
+  sg.kb = static_cast<int>(u % nkv);
+  const long long rest = u1 - u;
+  sg.ke = rest < nkv - sg.kb ? sg.kb + static_cast<int>(rest) : nkv;
+  u += sg.ke - sg.kb;
+  return true;
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out, int Lq, int Lk,
-                   int dh, float scale_log2, unsigned int* err, int debug_flags) {
+                   int dh, float scale_log2, unsigned int* err, int debug_flags, int qpairs, int items,
+                   float* __restrict__ ws, unsigned int* flags) {
   constexpr int BN = C::BN, NQ = C::NQ, STAGES = C::STAGES, NCH = C::NCH, NCHV = C::NCHV, DHP = C::DHP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -172,12 +201,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.y;
-  const int q0 = blockIdx.x * (BM * NQ);
   const int nkv = (Lk + BN - 1) / BN;
+  const long long U = static_cast<long long>(items) * nkv;
+  const long long u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
 
   if (threadIdx.x == 0) {
-    mbar_init(bars.q_full(), 1);
+    mbar_init(bars.q_full(0), 1);
+    mbar_init(bars.q_full(1), 1);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bars.k_full(s), 1);
       mbar_init(bars.v_full(s), 1);
@@ -192,6 +222,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     for (int t = 0; t < NQ; ++t) mbar_init(bars.fin() + 8 * t, 1);
     for (int i = 0; i < 8; ++i) mbar_init(bars.tok(i >> 2, i & 3), 1);
+    mbar_init(bars.q_empty(0), NQ);
+    mbar_init(bars.q_empty(1), NQ);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -217,31 +249,51 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       int issued[STAGES];
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) issued[s] = 0;
-      mbar_arrive_expect_tx(bars.q_full(), NQ * C::Q_TILE_BYTES);
-      for (int t = 0; t < NQ; ++t)
-        for (int c = 0; c < NCH; ++c)
-          tma_load_3d(sbase + C::Q_OFF + t * C::Q_TILE_BYTES + c * BM * 128, &tm_q, bars.q_full(), c * 64,
-                      q0 + t * BM, bh);
-      for (int j = 0; j < nkv; ++j) {
-        const int s = j % STAGES, round = j / STAGES;
-        if (j >= STAGES && !wait_bar(bars.kv_empty(s), (round - 1) & 1, abort_flag, err)) break;
-        mbar_arrive_expect_tx(bars.k_full(s), C::K_TILE_BYTES);
-        for (int c = 0; c < NCH; ++c)
-          tma_load_3d(sbase + C::K_OFF + s * C::K_TILE_BYTES + c * BN * 128, &tm_k, bars.k_full(s), c * 64,
-                      j * BN, bh);
-        issued[s] = round + 1;
-        if ((debug_flags & 1) && j == 0) break;  // test hook: V tile 0 never arrives
-        mbar_arrive_expect_tx(bars.v_full(s), C::V_TILE_BYTES);
-        for (int c = 0; c < NCHV; ++c)
-          tma_load_3d(sbase + C::V_OFF + s * C::V_TILE_BYTES + c * BN * 128, &tm_v, bars.v_full(s), c * 64,
-                      j * BN, bh);
+      long long u = u0;
+      Seg sg;
+      int nseg = 0, g = 0;  // segments started, K/V tiles issued (the ring position)
+      bool ok = true;
+      while (ok && next_seg(u, u1, nkv, sg)) {
+        const int bh = sg.it / qpairs, q0 = (sg.it % qpairs) * (BM * NQ);
+        // Q buffer qb is reused by the segment after next, once both tiles have issued their last
+        // S = Q K^T of the segment that used it.
+        const int qb = nseg % C::QBUF;
+        if (nseg >= C::QBUF && !wait_bar(bars.q_empty(qb), (nseg / C::QBUF - 1) & 1, abort_flag, err)) break;
+        mbar_arrive_expect_tx(bars.q_full(qb), NQ * C::Q_TILE_BYTES);
+        for (int t = 0; t < NQ; ++t)
+          for (int c = 0; c < NCH; ++c)
+            tma_load_3d(sbase + C::Q_OFF + (qb * NQ + t) * C::Q_TILE_BYTES + c * BM * 128, &tm_q, bars.q_full(qb),
+                        c * 64, q0 + t * BM, bh);
+        ++nseg;
+        for (int j = sg.kb; j < sg.ke; ++j, ++g) {
+          const int s = g % STAGES, round = g / STAGES;
+          if (g >= STAGES && !wait_bar(bars.kv_empty(s), (round - 1) & 1, abort_flag, err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bars.k_full(s), C::K_TILE_BYTES);
+          for (int c = 0; c < NCH; ++c)
+            tma_load_3d(sbase + C::K_OFF + s * C::K_TILE_BYTES + c * BN * 128, &tm_k, bars.k_full(s), c * 64,
+                        j * BN, bh);
+          issued[s] = round + 1;
+          if ((debug_flags & 1) && g == 0) {  // test hook: the first V tile never arrives
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bars.v_full(s), C::V_TILE_BYTES);
+          for (int c = 0; c < NCHV; ++c)
+            tma_load_3d(sbase + C::V_OFF + s * C::V_TILE_BYTES + c * BN * 128, &tm_v, bars.v_full(s), c * 64,
+                        j * BN, bh);
+        }
       }
       // Drain: every copy this thread issued has landed before the CTA may exit.
-      wait_bar(bars.q_full(), 0, abort_flag, err, false);
+      for (int k = nseg - 1; k >= 0 && k >= nseg - C::QBUF; --k)
+        wait_bar(bars.q_full(k % C::QBUF), (k / C::QBUF) & 1, abort_flag, err, false);
       for (int s = 0; s < STAGES; ++s)
         if (issued[s] > 0) {
           wait_bar(bars.k_full(s), (issued[s] - 1) & 1, abort_flag, err, false);
-          if (!(debug_flags & 1)) wait_bar(bars.v_full(s), (issued[s] - 1) & 1, abort_flag, err, false);
+          if (!((debug_flags & 1) && s == 0 && issued[s] == 1))
+            wait_bar(bars.v_full(s), (issued[s] - 1) & 1, abort_flag, err, false);
         }
     }
   } else if (warp == 1 || (NQ == 2 && warp == 2)) {
@@ -252,7 +304,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, C::NPV, true);
-      const uint32_t tq = sbase + C::Q_OFF + t * C::Q_TILE_BYTES;
+      uint32_t tq = sbase + C::Q_OFF + t * C::Q_TILE_BYTES;  // the current segment's Q buffer
       auto issue_qk = [&](int s) {  // S = Q K_s^T over the padded head dim
         const uint32_t d = tmem + t * C::TM_TILE + C::TM_S;
 #pragma unroll
@@ -273,53 +325,62 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           mma_ts(d, a + ks * 8, b, idesc_pv, (!first || ks > 0) ? 1u : 0u);
         }
       };
-      bool ok = wait_bar(bars.q_full(), 0, abort_flag, err);
-      // Two pending items per tile, issued in whichever order they become ready: S_jq = Q K_jq^T
-      // (needs K_jq, and the softmax's release of S_{jq-1} -- with P over S, the completion of
-      // P_{jq-1} V), and O += P_jp V_jp (needs P_jp and V_jp). P V goes first when both are
-      // ready: it frees the K/V stage the producer is waiting for.
-      int jq = 0, jp = 0;
-      long long t_idle = clock64();
-      uint32_t spins = 0;
-      while (ok && jp < nkv) {
-#ifdef SD_TRACE
-        if (jp < jq && mbar_test_wait(bars.p_full(t), jp & 1)) {
-          const int cta_ = blockIdx.x + gridDim.x * blockIdx.y;
-          if (cta_ < kTraceCtas && jp < kTraceIters && g_trace[cta_][warp][jp][2] == 0) g_trace[cta_][warp][jp][2] = clock64();
-        }
-#endif
-        const bool can_pv = jp < jq && mbar_test_wait(bars.p_full(t), jp & 1) &&
-                            mbar_test_wait(C::L_IN_V ? bars.v_ready(jp % STAGES) : bars.v_full(jp % STAGES),
-                                           (jp / STAGES) & 1);
-        if (can_pv) {
-          tc_fence_after();
-          issue_pv(jp % STAGES, jp == 0);
-          mma_commit(bars.o_done(t));
-          mma_commit(bars.kv_empty(jp % STAGES));
-          SD_TR(warp, jp, 1);
-          ++jp;
-          t_idle = clock64();
-          continue;
-        }
-        const bool can_qk = jq < nkv && mbar_test_wait(bars.k_full(jq % STAGES), (jq / STAGES) & 1) &&
-                            (jq == 0 || mbar_test_wait(C::P_SEP ? bars.s_free(t) : bars.o_done(t), (jq - 1) & 1));
-        if (can_qk) {
-          tc_fence_after();
-          issue_qk(jq % STAGES);
-          mma_commit(bars.s_full(t));
-          SD_TR(warp, jq, 0);
-          ++jq;
-          t_idle = clock64();
-          continue;
-        }
-        if ((++spins & 31u) == 0) {
-          if (*abort_flag) break;
-          if (clock64() - t_idle > kWaitLimitCycles) {
-            *abort_flag = 1;
-            atomicOr(err, sd::kDevErrTimeout);
-            break;
+      // Per segment, two pending items per tile, issued in whichever order they become ready:
+      // S_i = Q K_i^T (needs K_i, and the softmax's release of the previous S -- with P over S, the
+      // completion of the previous P V), and O += P_i V_i (needs P_i and V_i; the first P V of a
+      // segment overwrites O). P V goes first when both are ready: it frees the K/V stage the
+      // producer is waiting for. Barrier phases run on the CTA-wide K/V tile count gb + i.
+      long long u = u0;
+      Seg sg;
+      int nseg = 0, gb = 0;
+      bool ok = true;
+      while (ok && next_seg(u, u1, nkv, sg)) {
+        const int n = sg.ke - sg.kb;
+        const int qb = nseg % C::QBUF;
+        tq = sbase + C::Q_OFF + (qb * NQ + t) * C::Q_TILE_BYTES;
+        ok = wait_bar(bars.q_full(qb), (nseg / C::QBUF) & 1, abort_flag, err);
+        int jq = 0, jp = 0;
+        long long t_idle = clock64();
+        uint32_t spins = 0;
+        while (ok && jp < n) {
+          const int gp = gb + jp, gq = gb + jq;
+          const bool can_pv = jp < jq && mbar_test_wait(bars.p_full(t), gp & 1) &&
+                              mbar_test_wait(C::L_IN_V ? bars.v_ready(gp % STAGES) : bars.v_full(gp % STAGES),
+                                             (gp / STAGES) & 1);
+          if (can_pv) {
+            tc_fence_after();
+            issue_pv(gp % STAGES, jp == 0);
+            mma_commit(bars.o_done(t));
+            mma_commit(bars.kv_empty(gp % STAGES));
+            SD_TR(warp, gp, 1);
+            ++jp;
+            t_idle = clock64();
+            continue;
+          }
+          const bool can_qk = jq < n && mbar_test_wait(bars.k_full(gq % STAGES), (gq / STAGES) & 1) &&
+                              (gq == 0 || mbar_test_wait(C::P_SEP ? bars.s_free(t) : bars.o_done(t), (gq - 1) & 1));
+          if (can_qk) {
+            tc_fence_after();
+            issue_qk(gq % STAGES);
+            mma_commit(bars.s_full(t));
+            if (jq + 1 == n) mma_commit(bars.q_empty(qb));  // this tile is done reading the segment's Q
+            SD_TR(warp, gq, 0);
+            ++jq;
+            t_idle = clock64();
+            continue;
+          }
+          if (SD_MMA_IDLE_NS > 0) __nanosleep(SD_MMA_IDLE_NS);  // idle poll: leave issue slots to the softmax
+          if ((++spins & 31u) == 0) {
+            if (*abort_flag) ok = false;
+            else if (clock64() - t_idle > kWaitLimitCycles) {
+              *abort_flag = 1;
+              atomicOr(err, sd::kDevErrTimeout);
+              ok = false;
+            }
           }
         }
+        gb += n;
+        ++nseg;
       }
       // Drain: all tensor-core work issued by this thread completes before TMEM is released.
       const uint32_t fin = bars.fin() + 8 * t;
@@ -333,7 +394,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // Writes bf16 1.0 into column DH of every landed V tile (128-byte swizzled rows: the 16-byte
     // granule g of row r sits at granule g ^ (r % 8)), then hands the tile to the MMA issuer.
     constexpr int ch = C::DH / 64, byte = (C::DH % 64) * 2, g = byte >> 4, gb = byte & 15;
-    for (int j = 0; j < nkv; ++j) {
+    const int total = static_cast<int>(u1 - u0);  // K/V tiles this CTA streams
+    for (int j = 0; j < total; ++j) {
       const int s = j % STAGES;
       if (!__all_sync(0xffffffffu, wait_bar(bars.v_full(s), (j / STAGES) & 1, abort_flag, err))) break;
       uint8_t* vt = smem + C::V_OFF + s * C::V_TILE_BYTES + ch * BN * 128;
@@ -360,18 +422,25 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int row = quarter * 32 + lane;
     const uint32_t tbase = tmem + t * C::TM_TILE + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t tS = tbase + C::TM_S, tP = tbase + C::TM_P, tO = tbase + C::TM_O;
-    float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     const bool tr = lane == 0;
     const int trole = warp;
-    for (int j = 0; j < nkv; ++j) {
-      if (tr) SD_TR(trole, j, 0);
+    constexpr bool kPing = SD_PINGPONG && NQ == 2;
+    long long u = u0;
+    Seg sg;
+    int gi = 0;  // CTA-wide K/V tile count: the phase of every per-tile barrier
+    while (ok && next_seg(u, u1, nkv, sg)) {
+    const int bh = sg.it / qpairs, q0 = (sg.it % qpairs) * (BM * NQ);
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int j = sg.kb; j < sg.ke; ++j, ++gi) {
+      const bool first = j == sg.kb;  // O and l are (re)initialised by this segment's first P V
+      if (tr) SD_TR(trole, gi, 0);
       // warp-uniform outcome: the tcgen05 copies below are .sync.aligned
-      if (!__all_sync(0xffffffffu, wait_bar(bars.s_full(t), j & 1, abort_flag, err))) {
+      if (!__all_sync(0xffffffffu, wait_bar(bars.s_full(t), gi & 1, abort_flag, err))) {
         ok = false;
         break;
       }
-      if (tr) SD_TR(trole, j, 1);
+      if (tr) SD_TR(trole, gi, 1);
       tc_fence_after();
       float sv[BN];
 #pragma unroll
@@ -382,7 +451,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(r[i]);
       }
       tmem_wait_ld();
-      if (tr) SD_TR(trole, j, 2);
+      if (tr) SD_TR(trole, gi, 2);
       if constexpr (C::P_SEP) {  // S is in registers: the next S = Q K^T may overwrite it
         tc_fence_before();
         mbar_arrive(bars.s_free(t));
@@ -411,15 +480,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // Lazy rescale (always on the first tile). The decision is warp-uniform: the tcgen05 copies
       // of O and l below are .sync.aligned, and rescaling a row whose max barely moved is exact.
       const bool rescale = __any_sync(0xffffffffu, m_new > m_run + 8.0f);
-      if (tr) SD_TR(trole, j, 3);
+      if (tr) SD_TR(trole, gi, 3);
       const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
       if (rescale) m_run = m_new;
       // Ping-pong: the special-function unit of a sub-partition serves one tile's exp2 phase at a
       // time; the other tile's warp on it does its row max, P store and S load meanwhile. Tile 0
       // goes first; each warp hands the token to its partner (same sub-partition) after its exps.
-      constexpr bool kPing = SD_PINGPONG && NQ == 2;
-      if (kPing && (t == 1 || j > 0)) {
-        if (!__all_sync(0xffffffffu, wait_bar(bars.tok(t, quarter), (t == 1 ? j : j - 1) & 1, abort_flag, err))) {
+      if (kPing && (t == 1 || gi > 0)) {
+        if (!__all_sync(0xffffffffu, wait_bar(bars.tok(t, quarter), (t == 1 ? gi : gi - 1) & 1, abort_flag, err))) {
           ok = false;
           break;
         }
@@ -428,45 +496,34 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       uint32_t pk[BN / 2];
       float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-      for (int b = 0; b < BN / 32; ++b) {
-        // 16 column pairs at a time: all arguments, then all exponentials, then the packing, so
-        // that many independent special-function operations are in flight per warp.
-        float x[32];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          fma2(x[2 * i], x[2 * i + 1], sv[32 * b + 2 * i], sv[32 * b + 2 * i + 1], scale_log2, scale_log2, neg_m,
-               neg_m);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if ((i & 7) < C::POLY_PAIRS) {
-            exp2_poly2(x[2 * i], x[2 * i + 1], x[2 * i], x[2 * i + 1]);
-          } else {
-            x[2 * i] = ex2_approx(x[2 * i]);
-            x[2 * i + 1] = ex2_approx(x[2 * i + 1]);
-          }
+      for (int i = 0; i < BN / 2; ++i) {
+        float x0, x1;
+        fma2(x0, x1, sv[2 * i], sv[2 * i + 1], scale_log2, scale_log2, neg_m, neg_m);  // s * scale * log2e - m
+        if ((i & 7) < C::POLY_PAIRS) {
+          exp2_poly2(x0, x1, x0, x1);
+        } else {
+          x0 = ex2_approx(x0);
+          x1 = ex2_approx(x1);
         }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x[2 * i], x[2 * i + 1]);
-          pk[16 * b + i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
-        }
+        if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x0, x1);
+        pk[i] = pack_bf16x2(x0, x1);
       }
       if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
       if (kPing) {
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
       }
-      if (tr) SD_TR(trole, j, 4);
-      // P_{j-1} V (and the O it accumulates) must be complete before P_j and O are touched.
-      if (C::P_SEP && j > 0) {
-        if (!__all_sync(0xffffffffu, wait_bar(bars.o_done(t), (j - 1) & 1, abort_flag, err))) {
+      if (tr) SD_TR(trole, gi, 4);
+      // The previous P V (and the O it accumulates) must be complete before P and O are touched.
+      if (C::P_SEP && gi > 0) {
+        if (!__all_sync(0xffffffffu, wait_bar(bars.o_done(t), (gi - 1) & 1, abort_flag, err))) {
           ok = false;
           break;
         }
         tc_fence_after();
       }
-      if (tr) SD_TR(trole, j, 5);
-      if (rescale && j > 0) {
+      if (tr) SD_TR(trole, gi, 5);
+      if (rescale && !first) {
 #pragma unroll
         for (int c = 0; c < C::NPV / 16; ++c) {  // O columns, the row-sum column DH among them
           const uint32_t addr = tO + c * 16;
@@ -488,33 +545,88 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bars.p_full(t));
-      if (tr) SD_TR(trole, j, 6);
+      if (tr) SD_TR(trole, gi, 6);
     }
-    if (ok && __all_sync(0xffffffffu, wait_bar(bars.o_done(t), (nkv - 1) & 1, abort_flag, err))) {
-      tc_fence_after();
-      const int qrow = q0 + t * BM + row;
-      float lsum = l_run;
-      uint32_t packed[DHP / 2];
-      float ov[C::NPV];
+    if (!ok || !__all_sync(0xffffffffu, wait_bar(bars.o_done(t), (gi - 1) & 1, abort_flag, err))) {
+      ok = false;
+      break;
+    }
+    // ------------------------------------------------ epilogue of the segment (one row per thread)
+    tc_fence_after();
+    float ov[C::NPV];
 #pragma unroll
-      for (int c = 0; c < C::NPV / 16; ++c) {
-        uint32_t r[16];
-        tmem_ld16(tO + c * 16, r);
-        tmem_wait_ld();
+    for (int c = 0; c < C::NPV / 16; ++c) {
+      uint32_t r[16];
+      tmem_ld16(tO + c * 16, r);
+      tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) ov[c * 16 + i] = __uint_as_float(r[i]);
+      for (int i = 0; i < 16; ++i) ov[c * 16 + i] = __uint_as_float(r[i]);
+    }
+    float lsum = C::L_IN_V ? ov[C::DH] : l_run;
+    const int slot_row = t * BM + row;
+    if (sg.kb > 0) {
+      // Tail piece of an item split with the previous CTA: hand raw O, m and l to it.
+      float* slot = ws + static_cast<size_t>(blockIdx.x - 1) * C::SLOT_FLOATS;
+      float4* dst = reinterpret_cast<float4*>(slot + static_cast<size_t>(slot_row) * C::NPV);
+#pragma unroll
+      for (int i = 0; i < C::NPV / 4; ++i) dst[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
+      float2* ml = reinterpret_cast<float2*>(slot + NQ * BM * C::NPV) + slot_row;
+      *ml = make_float2(m_run, lsum);
+      __threadfence();
+      atomicAdd(flags + blockIdx.x - 1, 1u);
+      continue;
+    }
+    if (sg.ke < nkv) {
+      // Head piece: wait for the tail (the next CTA processed it at the start of its range), merge.
+      float* slot = ws + static_cast<size_t>(blockIdx.x) * C::SLOT_FLOATS;
+      volatile unsigned int* f = flags + blockIdx.x;
+      const long long w0 = clock64();
+      bool got = true;
+      for (uint32_t it = 0; *f < static_cast<unsigned>(NQ * BM); ++it) {
+        __nanosleep(64);
+        if ((it & 63u) == 63u && (*abort_flag || clock64() - w0 > kWaitLimitCycles)) {
+          if (!*abort_flag) {
+            *abort_flag = 1;
+            atomicOr(err, sd::kDevErrTimeout);
+          }
+          got = false;
+          break;
+        }
       }
-      if constexpr (C::L_IN_V) lsum = ov[C::DH];
-      const float inv_l = 1.0f / lsum;
-#pragma unroll
-      for (int i = 0; i < DHP / 2; ++i) packed[i] = pack_bf16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l);
-      if (qrow < Lq) {
-        uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * Lq + qrow) * dh);
-        const int n16 = dh / 8;  // 16-byte groups of 8 bf16
-#pragma unroll
-        for (int i = 0; i < DHP / 8; ++i)
-          if (i < n16) dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+      if (!got) {
+        ok = false;
+        break;
       }
+      __threadfence();
+      const float4* src = reinterpret_cast<const float4*>(slot + static_cast<size_t>(slot_row) * C::NPV);
+      const float2 ml = reinterpret_cast<const float2*>(slot + NQ * BM * C::NPV)[slot_row];
+      const float m_all = fmaxf(m_run, ml.x);
+      const float a_h = ex2_approx(m_run - m_all), a_t = ex2_approx(ml.x - m_all);
+#pragma unroll
+      for (int i = 0; i < C::NPV / 4; ++i) {
+        const float4 o4 = src[i];
+        ov[4 * i] = ov[4 * i] * a_h + o4.x * a_t;
+        ov[4 * i + 1] = ov[4 * i + 1] * a_h + o4.y * a_t;
+        ov[4 * i + 2] = ov[4 * i + 2] * a_h + o4.z * a_t;
+        ov[4 * i + 3] = ov[4 * i + 3] * a_h + o4.w * a_t;
+      }
+      lsum = C::L_IN_V ? ov[C::DH] : lsum * a_h + ml.y * a_t;
+      // consumed: the last of the 2 * NQ * 128 arrivals (tail writers, then these readers) resets
+      // the flag for the next launch
+      if (atomicAdd(flags + blockIdx.x, 1u) == static_cast<unsigned>(2 * NQ * BM - 1)) atomicExch(flags + blockIdx.x, 0u);
+    }
+    const int qrow = q0 + t * BM + row;
+    const float inv_l = 1.0f / lsum;
+    uint32_t packed[DHP / 2];
+#pragma unroll
+    for (int i = 0; i < DHP / 2; ++i) packed[i] = pack_bf16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l);
+    if (qrow < Lq) {
+      uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * Lq + qrow) * dh);
+      const int n16 = dh / 8;  // 16-byte groups of 8 bf16
+#pragma unroll
+      for (int i = 0; i < DHP / 8; ++i)
+        if (i < n16) dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+    }
     }
   }
   tc_fence_before();
@@ -555,6 +667,47 @@ sd_status make_map(CUtensorMap* map, const void* ptr, int64_t dh, int64_t rows, 
 
 int g_debug_flags = 0;
 
+// Per-device hand-off workspace of the persistent schedule (slots of split items + their flags).
+// Allocated on first need and grown, never shrunk; flags start at zero and every launch leaves them
+// at zero. Launches of sd_attention that run concurrently on one device (different streams) must not
+// both split items: they would share the slots.
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+Workspace g_ws[64];
+std::mutex g_ws_mu;
+
+sd_status workspace(size_t bytes, cudaStream_t s, void** out) {
+  int dev = 0;
+  sd_status st = sd::cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st != SD_OK) return st;
+  if (dev >= 64) return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention: device index >= 64");
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  Workspace& w = g_ws[dev];
+  if (w.bytes < bytes) {
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(s, &cap);
+    if (cap != cudaStreamCaptureStatusNone)
+      return sd::fail(SD_ERR_CUDA, "sd_attention: the split-item workspace (%zu bytes) must be allocated before "
+                                   "stream capture; run the same shape once outside the capture", bytes);
+    if (w.ptr) {
+      st = sd::cuda_check(cudaDeviceSynchronize(), "cudaDeviceSynchronize(workspace growth)");
+      if (st == SD_OK) st = sd::cuda_check(cudaFree(w.ptr), "cudaFree(workspace)");
+      w.ptr = nullptr;
+      w.bytes = 0;
+      if (st != SD_OK) return st;
+    }
+    st = sd::cuda_check(cudaMalloc(&w.ptr, bytes), "cudaMalloc(workspace)");
+    if (st != SD_OK) return st;
+    st = sd::cuda_check(cudaMemset(w.ptr, 0, bytes), "cudaMemset(workspace)");
+    if (st != SD_OK) return st;
+    w.bytes = bytes;
+  }
+  *out = w.ptr;
+  return SD_OK;
+}
+
 template <class C>
 sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t BH, int64_t Lq, int64_t Lk,
                  int64_t dh, float scale, cudaStream_t s) {
@@ -577,11 +730,28 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
     if (st != SD_OK) return st;
     smem_set.fetch_or(bit, std::memory_order_acq_rel);
   }
-  const dim3 grid(static_cast<unsigned>((Lq + BM * C::NQ - 1) / (BM * C::NQ)), static_cast<unsigned>(BH));
+  // Persistent grid: one CTA per SM (shared memory admits one), each owning an equal share of the
+  // items x K/V-tiles units; items split between two CTAs hand over through the workspace.
+  const int64_t qpairs = (Lq + BM * C::NQ - 1) / (BM * C::NQ);
+  const int64_t items = BH * qpairs;
+  const int64_t nkv = (Lk + C::BN - 1) / C::BN;
+  const int64_t G = std::min<int64_t>(sd::sm_count(), items);
+  if (items > 0x7fffffff || items * nkv > (int64_t(1) << 40))
+    return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention: too many tiles");
+  float* ws = nullptr;
+  unsigned int* flags = nullptr;
+  if (G < items && nkv > 1) {
+    const size_t fbytes = (static_cast<size_t>(G) * C::SLOT_FLOATS * sizeof(float) + 255) / 256 * 256;
+    void* p = nullptr;
+    st = workspace(fbytes + static_cast<size_t>(G) * sizeof(unsigned int), s, &p);
+    if (st != SD_OK) return st;
+    ws = static_cast<float*>(p);
+    flags = reinterpret_cast<unsigned int*>(static_cast<char*>(p) + fbytes);
+  }
   const float scale_log2 = scale * 1.4426950408889634f;
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, s>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), static_cast<int>(Lq),
-                                                static_cast<int>(Lk), static_cast<int>(dh), scale_log2, err,
-                                                g_debug_flags);
+  kern<<<static_cast<unsigned>(G), C::THREADS, C::SMEM_BYTES, s>>>(
+      mq, mk, mv, static_cast<__nv_bfloat16*>(o), static_cast<int>(Lq), static_cast<int>(Lk), static_cast<int>(dh),
+      scale_log2, err, g_debug_flags, static_cast<int>(qpairs), static_cast<int>(items), ws, flags);
   return sd::cuda_check(cudaGetLastError(), "sd_attention launch");
 }
 
@@ -597,8 +767,8 @@ extern "C" sd_status sd_attention(const void* q, const void* k, const void* v, v
   if (Lk == 0) return sd::fail(SD_ERR_INVALID_ARG, "sd_attention: Lk must be >= 1 when Lq >= 1");
   if (!q || !k || !v || !o) return sd::fail(SD_ERR_INVALID_ARG, "sd_attention: null pointer");
   const int64_t BH = B * heads;
-  if (BH > 65535 || Lq > (int64_t(1) << 30) || Lk > (int64_t(1) << 30))
-    return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention: B*heads must be <= 65535 and L <= 2^30");
+  if (BH > (int64_t(1) << 31) - 1 || Lq > (int64_t(1) << 30) || Lk > (int64_t(1) << 30))
+    return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention: B*heads must be < 2^31 and L <= 2^30");
   if (!sd::aligned16(q) || !sd::aligned16(k) || !sd::aligned16(v) || !sd::aligned16(o))
     return sd::fail(SD_ERR_MISALIGNED, "sd_attention: q, k, v and o must be 16-byte aligned");
   const int64_t qbytes = BH * Lq * dh * 2, kvbytes = BH * Lk * dh * 2;
