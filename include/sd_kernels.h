@@ -84,6 +84,33 @@ sd_status sd_attention(const void* q, const void* k, const void* v, void* o,
                        void* stream);
 
 /*
+ * sd_attention_noalloc -- the same computation, arguments, layouts and errors as sd_attention, for
+ * callers that cannot allocate device memory. (The source pages have no counterpart: this is an
+ * interface of this library.)
+ *
+ * Why it exists: sd_attention allocates a scratch workspace with cudaMalloc the first time a shape
+ * splits a query-tile item between two CTAs, and grows it when a later shape needs more. That is not
+ * possible for every caller: code that is being captured into a CUDA graph may not call cudaMalloc,
+ * a framework that owns all device memory through its own allocator may forbid outside
+ * allocations, and a latency-critical loop cannot absorb the device synchronisation that
+ * cudaMalloc and cudaFree imply. This entry point never calls cudaMalloc, cudaFree or any
+ * allocating routine: its scratch is a 16 MiB file-scope device array that every GPU loading the
+ * library holds until the process exits (enough for every head dim this library supports on up
+ * to 148 SMs). A shape whose scratch would exceed 16 MiB is rejected with SD_ERR_UNSUPPORTED and
+ * nothing is launched.
+ *
+ *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress); make
+ *    that first call before any stream capture on that device.
+ *  - Every call uses the same array, which keeps the previous call's contents; each call clears
+ *    the part that must start at zero with an asynchronous memset on `stream` before its kernel.
+ *  - Calls whose executions overlap on the GPU (different streams, no ordering between them) race
+ *    on the array and produce wrong results; order them on one stream or with events.
+ */
+sd_status sd_attention_noalloc(const void* q, const void* k, const void* v, void* o,
+                               int64_t B, int64_t heads, int64_t Lq, int64_t Lk, int64_t dh, float scale,
+                               void* stream);
+
+/*
  * Guided DDIM step. Guidance from "从零实现扩散模型推理引擎：Rust + wgpu 的 GPU 加速图像生成架构" §7 and
  * "本地部署扩散模型架构与底层运行原理深度解析" (示例说明): g = eps_u + w * (eps_c - eps_u), where eps_u and
  * eps_c are the unconditional and conditional halves of the UNet output (batch order

@@ -48,11 +48,12 @@ def lib() -> ctypes.CDLL:
         i64, f32, f64, vp, c_int = ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_void_p, ctypes.c_int
         L.sd_group_norm.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
         L.sd_attention.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
+        L.sd_attention_noalloc.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
         L.sd_cfg_ddim_step.argtypes = [vp, vp, vp, vp, i64, f32, f64, f64, vp]
         L.sd_device_status.argtypes = [vp, c_int]
         L.sd_debug_set_fault.argtypes = [c_int]
         L.sd_debug_set_fault.restype = None
-        for f in ("sd_group_norm", "sd_attention", "sd_cfg_ddim_step", "sd_device_status"):
+        for f in ("sd_group_norm", "sd_attention", "sd_attention_noalloc", "sd_cfg_ddim_step", "sd_device_status"):
             getattr(L, f).restype = c_int
         L.sd_status_string.argtypes = [c_int]
         L.sd_status_string.restype = ctypes.c_char_p
@@ -125,6 +126,27 @@ def sd_attention(q, k, v, scale: float | None = None, out=None):
         scale = 1.0 / math.sqrt(dh)
     _check("sd_attention", lib().sd_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hh, Lq,
                                               k.shape[2], dh, scale, _stream(q)))
+    return out
+
+
+def sd_attention_noalloc(q, k, v, scale: float | None = None, out=None):
+    """sd_attention without any device allocation by the library (fixed 16 MiB scratch instead).
+
+    For callers that cannot let a library call cudaMalloc: inside CUDA-graph capture, under a
+    framework that owns all device memory, or in loops that cannot absorb cudaMalloc's implicit
+    synchronisation. Pass ``out`` to avoid the allocation of the output tensor as well. Calls that
+    overlap on the GPU race on the shared scratch.
+    """
+    import torch
+    if out is None:
+        out = torch.empty_like(q)
+    _require_cuda(q, k, v, out)
+    B, Hh, Lq, dh = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(dh)
+    _check("sd_attention_noalloc", lib().sd_attention_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                              out.data_ptr(), B, Hh, Lq, k.shape[2], dh, scale,
+                                                              _stream(q)))
     return out
 
 

@@ -708,9 +708,38 @@ sd_status workspace(size_t bytes, cudaStream_t s, void** out) {
   return SD_OK;
 }
 
+// Fixed scratch of sd_attention_noalloc: a file-scope device array, so that entry point never
+// allocates. Every device that loads the library holds it until the process exits. Zero at module
+// load; each call clears the hand-off flags it uses before its launch.
+constexpr size_t kFixedScratchBytes = size_t(16) << 20;
+__device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchBytes];
+void* g_fixed_addr[64] = {};
+std::mutex g_fixed_mu;
+
+// Device address of g_fixed_scratch on the current device. The name of the array in host code is a
+// host-side stand-in, not a device address, so it is resolved once per device with that device
+// current and cached.
+sd_status fixed_scratch(void** out) {
+  int dev = 0;
+  sd_status st = sd::cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st != SD_OK) return st;
+  if (dev >= 64) return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention_noalloc: device index >= 64");
+  std::lock_guard<std::mutex> lock(g_fixed_mu);
+  if (!g_fixed_addr[dev]) {
+    void* p = nullptr;
+    st = sd::cuda_check(cudaGetSymbolAddress(&p, g_fixed_scratch), "cudaGetSymbolAddress(fixed scratch)");
+    if (st != SD_OK) return st;
+    g_fixed_addr[dev] = p;
+  }
+  *out = g_fixed_addr[dev];
+  return SD_OK;
+}
+
+// `fixed` selects the caller-side contract of sd_attention_noalloc: scratch from g_fixed_scratch
+// instead of the growable workspace, with its flags cleared on the stream first.
 template <class C>
 sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t BH, int64_t Lq, int64_t Lk,
-                 int64_t dh, float scale, cudaStream_t s) {
+                 int64_t dh, float scale, cudaStream_t s, bool fixed = false) {
   CUtensorMap mq, mk, mv;
   sd_status st = make_map(&mq, q, dh, Lq, BH, BM);
   if (st == SD_OK) st = make_map(&mk, k, dh, Lk, BH, C::BN);
@@ -742,8 +771,19 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
   unsigned int* flags = nullptr;
   if (G < items && nkv > 1) {
     const size_t fbytes = (static_cast<size_t>(G) * C::SLOT_FLOATS * sizeof(float) + 255) / 256 * 256;
+    const size_t need = fbytes + static_cast<size_t>(G) * sizeof(unsigned int);
     void* p = nullptr;
-    st = workspace(fbytes + static_cast<size_t>(G) * sizeof(unsigned int), s, &p);
+    if (fixed) {
+      if (need > kFixedScratchBytes)
+        return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention_noalloc: this shape needs %zu bytes of scratch; the fixed "
+                                            "buffer holds %zu", need, kFixedScratchBytes);
+      st = fixed_scratch(&p);
+      if (st != SD_OK) return st;
+      st = sd::cuda_check(cudaMemsetAsync(static_cast<char*>(p) + fbytes, 0, need - fbytes, s),
+                          "cudaMemsetAsync(fixed scratch flags)");
+    } else {
+      st = workspace(need, s, &p);
+    }
     if (st != SD_OK) return st;
     ws = static_cast<float*>(p);
     flags = reinterpret_cast<unsigned int*>(static_cast<char*>(p) + fbytes);
@@ -757,8 +797,10 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
 
 }  // namespace
 
-extern "C" sd_status sd_attention(const void* q, const void* k, const void* v, void* o, int64_t B, int64_t heads,
-                                  int64_t Lq, int64_t Lk, int64_t dh, float scale, void* stream) {
+namespace {
+
+sd_status attention_impl(const void* q, const void* k, const void* v, void* o, int64_t B, int64_t heads, int64_t Lq,
+                         int64_t Lk, int64_t dh, float scale, void* stream, bool fixed) {
   if (B < 0 || heads < 0 || Lq < 0 || Lk < 0) return sd::fail(SD_ERR_INVALID_ARG, "sd_attention: negative size");
   if (dh != 40 && dh != 64 && dh != 80 && dh != 160)
     return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention: head dim %lld not in {40, 64, 80, 160}", (long long)dh);
@@ -777,18 +819,33 @@ extern "C" sd_status sd_attention(const void* q, const void* k, const void* v, v
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (Lk <= 96) {  // short key sequence (the 77-token text context): one 96-key tile, no online rescale
     switch (dh) {
-      case 40: return launch<Cfg<40, 96, 2, 2, true, true, 0>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
-      case 64: return launch<Cfg<64, 96, 2, 2, true, false>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
-      case 80: return launch<Cfg<80, 96, 2, 2, true, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
+      case 40: return launch<Cfg<40, 96, 2, 2, true, true, 0>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+      case 64: return launch<Cfg<64, 96, 2, 2, true, false>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+      case 80: return launch<Cfg<80, 96, 2, 2, true, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
       default: break;  // dh = 160 already uses 64-key tiles
     }
   }
   switch (dh) {
-    case 40: return launch<Cfg<40, 128, 2, SD_STAGES_SMALL, true, true, 0>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
-    case 64: return launch<Cfg<64, 128, 2, SD_STAGES_SMALL, true, false>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
-    case 80: return launch<Cfg<80, 128, 2, 2, false, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
-    default: return launch<Cfg<160, 64, 1, 3, true, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s);
+    case 40: return launch<Cfg<40, 128, 2, SD_STAGES_SMALL, true, true, 0>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+    case 64: return launch<Cfg<64, 128, 2, SD_STAGES_SMALL, true, false>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+    case 80: return launch<Cfg<80, 128, 2, 2, false, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+    default: return launch<Cfg<160, 64, 1, 3, true, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
   }
+}
+
+}  // namespace
+
+extern "C" sd_status sd_attention(const void* q, const void* k, const void* v, void* o, int64_t B, int64_t heads,
+                                  int64_t Lq, int64_t Lk, int64_t dh, float scale, void* stream) {
+  return attention_impl(q, k, v, o, B, heads, Lq, Lk, dh, scale, stream, false);
+}
+
+// Same computation for callers that cannot allocate device memory (see sd_kernels.h): scratch comes
+// from the fixed file-scope array; the first call on a device resolves its address.
+extern "C" sd_status sd_attention_noalloc(const void* q, const void* k, const void* v, void* o, int64_t B,
+                                          int64_t heads, int64_t Lq, int64_t Lk, int64_t dh, float scale,
+                                          void* stream) {
+  return attention_impl(q, k, v, o, B, heads, Lq, Lk, dh, scale, stream, true);
 }
 
 // Test hook (declared in sd_kernels.h): bit 0 makes the next attention launches skip their first
