@@ -301,6 +301,7 @@ def bench_ours(args, rank, world, dev):
                 "algorithmic_flops_per_launch": attention_flops(s_self)}
 
     e2e = bench_e2e(args, sdk, sets[0], g, a_t, a_p, wl.guidance, flops_step, world, dev)
+    extra = {} if args.no_extra else bench_extra(sdk, dev, hbm)
     out = {
         "metric": "attention TFLOP/s over the UNet hot-path step (GroupNorm + self-attn + cross-attn + CFG/DDIM)",
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -317,10 +318,72 @@ def bench_ours(args, rank, world, dev):
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": 4 * args.steps,
+        "extra": extra,
         "clocks": clk.summary(),
         "host_wall_s_timed_region": wall,
     }
     return out, sets
+
+
+def _graph_time_us(fn, n, dev):
+    """Average device time of fn() over n launches captured in one CUDA graph (after warm-up)."""
+    import torch
+    for _ in range(3):
+        fn(0)
+    torch.cuda.synchronize()
+    st = torch.cuda.Stream(device=dev)
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr, stream=st):
+        for i in range(n):
+            fn(i)
+    gr.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    gr.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / n
+
+
+def bench_extra(sdk, dev, hbm):
+    """Labelled extras, not the headline: the 20-step guided DDIM loop of the batched-serving
+    workload (one CUDA graph), and a size sweep of GroupNorm and CFG+DDIM up to buffers far larger
+    than L2 that shows the asymptotic HBM bandwidth of these small-shape kernels."""
+    import torch
+    out = {}
+    lat = si.WORKLOADS[5].latent
+    x = torch.randn(lat, device=dev)
+    eps = [(torch.randn(lat, device=dev), torch.randn(lat, device=dev)) for _ in range(20)]
+    sched = sdk.ddim_schedule(20)
+
+    def loop(_):
+        for (t, a_t, a_p), (eu, ec) in zip(sched, eps):
+            sdk.sd_cfg_ddim_step(x, eu, ec, 7.5, a_t, a_p, out=x)
+    us = _graph_time_us(loop, 5, dev)
+    n = int(np.prod(lat))
+    out["cfg_ddim_20_steps_serving"] = {"shape": list(lat), "us_per_loop": us, "us_per_step": us / 20,
+                                        "GB/s": 20 * 16 * n / (us * 1e-6) / 1e9}
+    sweep = []
+    for (B, C, H, W) in [(2, 320, 64, 64), (8, 320, 96, 96), (16, 640, 64, 64), (16, 320, 128, 128)]:
+        xs = [torch.randn(B, C, H, W, device=dev) for _ in range(2)]
+        gm, bt = torch.ones(C, device=dev), torch.zeros(C, device=dev)
+        ys = [torch.empty_like(t) for t in xs]
+        us = _graph_time_us(lambda i: sdk.sd_group_norm(xs[i % 2], gm, bt, 32, 1e-5, out=ys[i % 2]), 20, dev)
+        gbs = 8 * B * C * H * W / (us * 1e-6) / 1e9
+        sweep.append({"kernel": "group_norm", "shape": [B, C, H, W], "MB": 8 * B * C * H * W / 1e6, "us": us,
+                      "GB/s": gbs, "frac_hbm": gbs / hbm})
+        del xs, ys
+    for n in [1 << 20, 1 << 24, 1 << 26]:
+        a, u, c, o = (torch.randn(n, device=dev) for _ in range(4))
+        us = _graph_time_us(lambda i: sdk.sd_cfg_ddim_step(a, u, c, 7.5, 0.3, 0.5, out=o), 20, dev)
+        gbs = 16 * n / (us * 1e-6) / 1e9
+        sweep.append({"kernel": "cfg_ddim", "elements": n, "MB": 16 * n / 1e6, "us": us, "GB/s": gbs,
+                      "frac_hbm": gbs / hbm})
+        del a, u, c, o
+    out["bandwidth_sweep"] = sweep
+    torch.cuda.empty_cache()
+    return out
 
 
 def bench_e2e(args, sdk, S, g, a_t, a_p, w, flops_step, world, dev):
@@ -457,6 +520,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the labelled DDIM-loop and bandwidth-sweep extras")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -66,6 +66,10 @@ __device__ long long g_trace[kTraceCtas][12][kTraceIters][kTraceSlots];
 #define SD_PINGPONG 1  // alternate the two query tiles' exp2 phases on each SM sub-partition
 #endif
 
+#ifndef SD_SETMAXNREG
+#define SD_SETMAXNREG 0  // 1: move registers from the helper warpgroup to the softmax ones (measured slower)
+#endif
+
 #ifndef SD_MMA_IDLE_NS
 #define SD_MMA_IDLE_NS 0  // backoff of the MMA issuers' idle poll, in ns (0 = spin)
 #endif
@@ -122,6 +126,10 @@ struct Cfg {
   static constexpr int SOFT_WARP0 = 4;
   static constexpr int NUM_WARPS = 4 + 4 * NQ;
   static constexpr int THREADS = 32 * NUM_WARPS;
+  // Register split for NQ = 2 (setmaxnreg): the helper warpgroup drops to 40 per thread and the two
+  // softmax warpgroups rise to 232; 128 * 40 + 256 * 232 equals the launch budget of 168 x 384.
+  static constexpr int REG_HELPER = 40, REG_SOFT = 232;
+  static_assert(NQ != 2 || 128 * REG_HELPER + 256 * REG_SOFT <= 168 * 384, "register split exceeds the launch budget");
   // Split-item hand-off slot: raw O (NPV fp32 per row) and (m, l) per row of the NQ tiles.
   static constexpr int SLOT_FLOATS = NQ * BM * (NPV + 2);
   // Of every 8 column pairs, this many take the FMA-pipe exp2 instead of the special-function unit.
@@ -151,7 +159,7 @@ struct Bars {
 
 // Bounded wait. Returns false if this CTA has aborted or the limit expired (then it raises the
 // CTA's abort flag and the device status word). `abortable = false` is for teardown drains.
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, unsigned int* err,
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, unsigned int* err,
                                       bool abortable = true) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
@@ -243,6 +251,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   if (warp < C::SOFT_WARP0) {
   // ==================================================================== helper warpgroup
+  if (SD_SETMAXNREG && NQ == 2) regs_dec<C::REG_HELPER>();  // registers move to the softmax warpgroups
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -415,6 +424,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   }
   } else {
   // ==================================================================== softmax warpgroups
+  if (SD_SETMAXNREG && NQ == 2) regs_inc<C::REG_SOFT>();
   {
     // ------------------------------------------------------------------ softmax warps
     const int t = (warp - C::SOFT_WARP0) >> 2;  // query tile of this warpgroup

@@ -175,6 +175,17 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Warpgroup-wide register reallocation; every warp of the warpgroup executes it. (No non-inlined
+// calls may follow in the raised region: the callee would be compiled for the launch budget.)
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" :: "n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" :: "n"(N));
+}
+
 // ---------------------------------------------------------------- math
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
