@@ -66,6 +66,10 @@ __device__ long long g_trace[kTraceCtas][12][kTraceIters][kTraceSlots];
 #define SD_PINGPONG 1  // alternate the two query tiles' exp2 phases on each SM sub-partition
 #endif
 
+#ifndef SD_CROSS_NQ
+#define SD_CROSS_NQ 2  // query tiles per CTA for key sequences of at most 96 tokens
+#endif
+
 #ifndef SD_SETMAXNREG
 #define SD_SETMAXNREG 0  // 1: move registers from the helper warpgroup to the softmax ones (measured slower)
 #endif
@@ -829,15 +833,15 @@ sd_status attention_impl(const void* q, const void* k, const void* v, void* o, i
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (Lk <= 96) {  // short key sequence (the 77-token text context): one 96-key tile, no online rescale
     switch (dh) {
-      case 40: return launch<Cfg<40, 96, 2, 2, true, true, 0>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-      case 64: return launch<Cfg<64, 96, 2, 2, true, false>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-      case 80: return launch<Cfg<80, 96, 2, 2, true, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+      case 40: return launch<Cfg<40, 96, SD_CROSS_NQ, 2, true, true, 0>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+      case 64: return launch<Cfg<64, 96, SD_CROSS_NQ, 2, true, false>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+      case 80: return launch<Cfg<80, 96, SD_CROSS_NQ, 2, true, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
       default: break;  // dh = 160 already uses 64-key tiles
     }
   }
   switch (dh) {
-    case 40: return launch<Cfg<40, 128, 2, SD_STAGES_SMALL, true, true, 0>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-    case 64: return launch<Cfg<64, 128, 2, SD_STAGES_SMALL, true, false>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+    case 40: return launch<Cfg<40, 128, 2, SD_STAGES_SMALL, true, true, 2>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+    case 64: return launch<Cfg<64, 128, 2, SD_STAGES_SMALL, true, false, 2>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
     case 80: return launch<Cfg<80, 128, 2, 2, false, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
     default: return launch<Cfg<160, 64, 1, 3, true, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
   }

@@ -193,22 +193,23 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-// Packed two-lane fp32 arithmetic (one instruction for two values).
+// Packed two-lane fp32 arithmetic (one instruction for two values), through the sm_100 float2
+// builtins so that the compiler keeps the operands in register pairs.
 __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
                                      float c1) {
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2,%3};\n\tmov.b64 rb, {%4,%5};\n\t"
-      "mov.b64 rc, {%6,%7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0,%1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+  const float2 r = __ffma2_rn(make_float2(a0, a1), make_float2(b0, b1), make_float2(c0, c1));
+  d0 = r.x;
+  d1 = r.y;
 }
 __device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2,%3};\n\tmov.b64 rb, {%4,%5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0,%1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+  const float2 r = __fadd2_rn(make_float2(a0, a1), make_float2(b0, b1));
+  d0 = r.x;
+  d1 = r.y;
 }
 __device__ __forceinline__ void sub2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2,%3};\n\tmov.b64 rb, {%4,%5};\n\t"
-      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0,%1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1) : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+  const float2 r = __ffma2_rn(make_float2(b0, b1), make_float2(-1.0f, -1.0f), make_float2(a0, a1));  // a - b
+  d0 = r.x;
+  d1 = r.y;
 }
 
 // 2^x for two values on the FMA pipe: x = n + f with n = round(x), f in [-1/2, 1/2] (Cody-Waite
