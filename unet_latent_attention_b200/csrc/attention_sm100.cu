@@ -49,7 +49,7 @@ using namespace sm100;
 
 #ifdef SD_TRACE
 // Tuning builds only: per-CTA phase timestamps of the first softmax warp and of the MMA warp.
-constexpr int kTraceCtas = 64, kTraceIters = 40, kTraceSlots = 8;
+constexpr int kTraceCtas = 64, kTraceIters = 40, kTraceSlots = 8, kTraceLast = kTraceIters - 1;
 __device__ long long g_trace[kTraceCtas][12][kTraceIters][kTraceSlots];
 #define SD_TR(role, j, slot)                                                                        \
   do {                                                                                              \
@@ -57,6 +57,7 @@ __device__ long long g_trace[kTraceCtas][12][kTraceIters][kTraceSlots];
     if (cta_ < kTraceCtas && (j) < kTraceIters) g_trace[cta_][role][j][slot] = clock64();           \
   } while (0)
 #else
+constexpr int kTraceLast = 0;
 #define SD_TR(role, j, slot) \
   do {                       \
   } while (0)
@@ -68,6 +69,14 @@ __device__ long long g_trace[kTraceCtas][12][kTraceIters][kTraceSlots];
 
 #ifndef SD_CROSS_NQ
 #define SD_CROSS_NQ 2  // query tiles per CTA for key sequences of at most 96 tokens
+#endif
+
+#ifndef SD_EXP_BLOCK
+#define SD_EXP_BLOCK 1  // column pairs per exp2 block (1 = pair by pair)
+#endif
+
+#ifndef SD_PING_SHORT
+#define SD_PING_SHORT 1  // ping-pong also for the single 96-key tile of short key sequences
 #endif
 
 #ifndef SD_SETMAXNREG
@@ -217,6 +226,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const long long U = static_cast<long long>(items) * nkv;
   const long long u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
 
+  if (threadIdx.x == 0) SD_TR(0, kTraceLast, 0);  // kernel entry (tuning builds only)
   if (threadIdx.x == 0) {
     mbar_init(bars.q_full(0), 1);
     mbar_init(bars.q_full(1), 1);
@@ -252,6 +262,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (threadIdx.x == 0) SD_TR(0, kTraceLast, 1);  // prologue done
 
   if (warp < C::SOFT_WARP0) {
   // ==================================================================== helper warpgroup
@@ -439,7 +450,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     bool ok = true;
     const bool tr = lane == 0;
     const int trole = warp;
-    constexpr bool kPing = SD_PINGPONG && NQ == 2;
+    constexpr bool kPing = SD_PINGPONG && NQ == 2 && (SD_PING_SHORT || BN == 128);
     long long u = u0;
     Seg sg;
     int gi = 0;  // CTA-wide K/V tile count: the phase of every per-tile barrier
@@ -509,18 +520,30 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const float neg_m = -m_run;
       uint32_t pk[BN / 2];
       float ls0 = 0.f, ls1 = 0.f;
+      // Exponentials in blocks of EB column pairs: all arguments, then all exp2 (special-function
+      // unit, or the FMA-pipe polynomial for POLY_PAIRS of every 8 pairs), then all packing, so
+      // that a warp keeps many independent exp2 in flight instead of waiting on each pair.
+      constexpr int EB = SD_EXP_BLOCK;
 #pragma unroll
-      for (int i = 0; i < BN / 2; ++i) {
-        float x0, x1;
-        fma2(x0, x1, sv[2 * i], sv[2 * i + 1], scale_log2, scale_log2, neg_m, neg_m);  // s * scale * log2e - m
-        if ((i & 7) < C::POLY_PAIRS) {
-          exp2_poly2(x0, x1, x0, x1);
-        } else {
-          x0 = ex2_approx(x0);
-          x1 = ex2_approx(x1);
+      for (int b = 0; b < BN / 2; b += EB) {
+        float x[2 * EB];
+#pragma unroll
+        for (int i = 0; i < EB; ++i)  // s * scale * log2(e) - m, two columns per instruction
+          fma2(x[2 * i], x[2 * i + 1], sv[2 * (b + i)], sv[2 * (b + i) + 1], scale_log2, scale_log2, neg_m, neg_m);
+#pragma unroll
+        for (int i = 0; i < EB; ++i) {
+          if (((b + i) & 7) < C::POLY_PAIRS) {
+            exp2_poly2(x[2 * i], x[2 * i + 1], x[2 * i], x[2 * i + 1]);
+          } else {
+            x[2 * i] = ex2_approx(x[2 * i]);
+            x[2 * i + 1] = ex2_approx(x[2 * i + 1]);
+          }
         }
-        if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x0, x1);
-        pk[i] = pack_bf16x2(x0, x1);
+#pragma unroll
+        for (int i = 0; i < EB; ++i) {
+          if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x[2 * i], x[2 * i + 1]);
+          pk[b + i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+        }
       }
       if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
       if (kPing) {
@@ -641,6 +664,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int i = 0; i < DHP / 8; ++i)
         if (i < n16) dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
     }
+    if (tr) SD_TR(trole, gi - 1, 7);  // segment epilogue done
     }
   }
   tc_fence_before();
