@@ -51,6 +51,34 @@ using namespace sm100;
 // Tuning builds only: per-CTA phase timestamps of the first softmax warp and of the MMA warp.
 constexpr int kTraceCtas = 64, kTraceIters = 40, kTraceSlots = 8, kTraceLast = kTraceIters - 1;
 __device__ long long g_trace[kTraceCtas][12][kTraceIters][kTraceSlots];
+__device__ unsigned long long g_span[1024][2];  // global-timer ns at CTA entry and exit
+__device__ unsigned long long g_span_seq[8][1024][2];  // the same per launch (launch index mod 8)
+__device__ unsigned int g_span_entries;
+__device__ unsigned int g_span_smid[1024];
+__device__ unsigned long long g_seg[1024][8];  // release of the grid dependency, then segment ends
+#define SD_SEG(slot)                                                                          \
+  do {                                                                                        \
+    if (blockIdx.x < 1024 && (slot) < 8) g_seg[blockIdx.x][slot] = gtimer();                  \
+  } while (0)
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+#define SD_SPAN(slot)                                                                \
+  do {                                                                               \
+    if (threadIdx.x == 0 && blockIdx.x < 1024) {                                     \
+      const unsigned long long t_ = gtimer();                                        \
+      if ((slot) == 0) span_launch_ = atomicAdd(&g_span_entries, 1u) / gridDim.x;    \
+      g_span[blockIdx.x][slot] = t_;                                                 \
+      if ((slot) == 0) {                                                             \
+        unsigned int sm_;                                                            \
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(sm_));                            \
+        g_span_smid[blockIdx.x] = sm_;                                               \
+      }                                                                              \
+      g_span_seq[span_launch_ & 7][blockIdx.x][slot] = t_;                           \
+    }                                                                                \
+  } while (0)
 #define SD_TR(role, j, slot)                                                                        \
   do {                                                                                              \
     const int cta_ = blockIdx.x + gridDim.x * blockIdx.y;                                          \
@@ -61,6 +89,21 @@ constexpr int kTraceLast = 0;
 #define SD_TR(role, j, slot) \
   do {                       \
   } while (0)
+#define SD_SPAN(slot) \
+  do {                \
+  } while (0)
+#define SD_SEG(slot) \
+  do {               \
+  } while (0)
+#endif
+#ifdef SD_TRACE
+#define SD_SPAN_DECL __shared__ unsigned int span_launch_
+#else
+#define SD_SPAN_DECL
+#endif
+
+#ifndef SD_EXP_BF16
+#define SD_EXP_BF16 0  // tuning: exp2 of bf16 pairs on the special-function unit (see the exp loop)
 #endif
 
 #ifndef SD_PINGPONG
@@ -121,7 +164,7 @@ struct Cfg {
   static constexpr int BAR_OFF = V_OFF + STAGES * V_TILE_BYTES;
   // q_full, k_full[S], v_full[S], v_ready[S], kv_empty[S], s_full[NQ], s_free[NQ], p_full[NQ], o_done[NQ],
   // fin[NQ], the exp tokens tok[2][4] of the two tiles' warps on each SM sub-partition, q_empty
-  static constexpr int NBARS = 2 + 4 * STAGES + 5 * NQ + 8 + 2;
+  static constexpr int NBARS = 2 + 4 * STAGES + 5 * NQ + 8 + 2 + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
   // TMEM columns of one query tile: S | P (if separate) | O (NPV columns, l at column DH)
@@ -168,6 +211,10 @@ struct Bars {
   __device__ uint32_t fin() const { return base + 8 * (2 + 4 * stages + 4 * nq); }
   __device__ uint32_t tok(int t, int q) const { return base + 8 * (2 + 4 * stages + 5 * nq + 4 * t + q); }
   __device__ uint32_t q_empty(int b) const { return base + 8 * (2 + 4 * stages + 5 * nq + 8 + b); }
+  // split-item hand-off: the tail piece's slot is written (all softmax threads), the head piece's
+  // slot may be read (the leader has seen the other CTA's flag)
+  __device__ uint32_t slot_written() const { return base + 8 * (2 + 4 * stages + 5 * nq + 10); }
+  __device__ uint32_t slot_ready() const { return base + 8 * (2 + 4 * stages + 5 * nq + 11); }
 };
 
 // Bounded wait. Returns false if this CTA has aborted or the limit expired (then it raises the
@@ -227,6 +274,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const long long u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
 
   if (threadIdx.x == 0) SD_TR(0, kTraceLast, 0);  // kernel entry (tuning builds only)
+  SD_SPAN_DECL;
+  SD_SPAN(0);
   if (threadIdx.x == 0) {
     mbar_init(bars.q_full(0), 1);
     mbar_init(bars.q_full(1), 1);
@@ -246,6 +295,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     for (int i = 0; i < 8; ++i) mbar_init(bars.tok(i >> 2, i & 3), 1);
     mbar_init(bars.q_empty(0), NQ);
     mbar_init(bars.q_empty(1), NQ);
+    mbar_init(bars.slot_written(), NQ * BM);
+    mbar_init(bars.slot_ready(), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -262,6 +313,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // Everything above touched only shared memory, tensor memory and the kernel parameters: it may
+  // overlap the end of the previous kernel on the stream. Global memory waits for that kernel.
+  sd::grid_dep_wait();
+  sd::grid_dep_launch();
+  if (threadIdx.x == 0) SD_SEG(0);
   if (threadIdx.x == 0) SD_TR(0, kTraceLast, 1);  // prologue done
 
   if (warp < C::SOFT_WARP0) {
@@ -349,62 +405,68 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           mma_ts(d, a + ks * 8, b, idesc_pv, (!first || ks > 0) ? 1u : 0u);
         }
       };
-      // Per segment, two pending items per tile, issued in whichever order they become ready:
-      // S_i = Q K_i^T (needs K_i, and the softmax's release of the previous S -- with P over S, the
-      // completion of the previous P V), and O += P_i V_i (needs P_i and V_i; the first P V of a
-      // segment overwrites O). P V goes first when both are ready: it frees the K/V stage the
-      // producer is waiting for. Barrier phases run on the CTA-wide K/V tile count gb + i.
-      long long u = u0;
-      Seg sg;
-      int nseg = 0, gb = 0;
+      // Two cursors over the CTA's K/V tiles, issued in whichever order they become ready:
+      // S_g = Q K_g^T (needs K_g, the segment's Q, and the softmax's release of the previous S --
+      // with P over S, the completion of the previous P V), and O += P_g V_g (needs P_g and V_g;
+      // the first P V of a segment overwrites O, which the softmax has read out before it stores
+      // that segment's first P). P V goes first when both are ready: it frees the K/V stage the
+      // producer is waiting for. The S cursor runs ahead into the next segment, so its first S
+      // overlaps the previous segment's last P V and epilogue. Barrier phases run on the
+      // CTA-wide K/V tile counts gq, gp.
+      long long uq = u0, up = u0;
+      Seg sq, sp;
+      bool have_q = next_seg(uq, u1, nkv, sq), have_p = next_seg(up, u1, nkv, sp);
+      int nseg_q = 0, jq = 0, jp = 0, gq = 0, gp = 0;
       bool ok = true;
-      while (ok && next_seg(u, u1, nkv, sg)) {
-        const int n = sg.ke - sg.kb;
-        const int qb = nseg % C::QBUF;
-        tq = sbase + C::Q_OFF + (qb * NQ + t) * C::Q_TILE_BYTES;
-        ok = wait_bar(bars.q_full(qb), (nseg / C::QBUF) & 1, abort_flag, err);
-        int jq = 0, jp = 0;
-        long long t_idle = clock64();
-        uint32_t spins = 0;
-        while (ok && jp < n) {
-          const int gp = gb + jp, gq = gb + jq;
-          const bool can_pv = jp < jq && mbar_test_wait(bars.p_full(t), gp & 1) &&
-                              mbar_test_wait(C::L_IN_V ? bars.v_ready(gp % STAGES) : bars.v_full(gp % STAGES),
-                                             (gp / STAGES) & 1);
-          if (can_pv) {
-            tc_fence_after();
-            issue_pv(gp % STAGES, jp == 0);
-            mma_commit(bars.o_done(t));
-            mma_commit(bars.kv_empty(gp % STAGES));
-            SD_TR(warp, gp, 1);
-            ++jp;
-            t_idle = clock64();
-            continue;
+      long long t_idle = clock64();
+      uint32_t spins = 0;
+      while (ok && have_p) {
+        const bool can_pv = gp < gq && mbar_test_wait(bars.p_full(t), gp & 1) &&
+                            mbar_test_wait(C::L_IN_V ? bars.v_ready(gp % STAGES) : bars.v_full(gp % STAGES),
+                                           (gp / STAGES) & 1);
+        if (can_pv) {
+          tc_fence_after();
+          issue_pv(gp % STAGES, jp == 0);
+          mma_commit(bars.o_done(t));
+          mma_commit(bars.kv_empty(gp % STAGES));
+          SD_TR(warp, gp, 1);
+          ++gp;
+          if (++jp == sp.ke - sp.kb) {
+            have_p = next_seg(up, u1, nkv, sp);
+            jp = 0;
           }
-          const bool can_qk = jq < n && mbar_test_wait(bars.k_full(gq % STAGES), (gq / STAGES) & 1) &&
-                              (gq == 0 || mbar_test_wait(C::P_SEP ? bars.s_free(t) : bars.o_done(t), (gq - 1) & 1));
-          if (can_qk) {
-            tc_fence_after();
-            issue_qk(gq % STAGES);
-            mma_commit(bars.s_full(t));
-            if (jq + 1 == n) mma_commit(bars.q_empty(qb));  // this tile is done reading the segment's Q
-            SD_TR(warp, gq, 0);
-            ++jq;
-            t_idle = clock64();
-            continue;
+          t_idle = clock64();
+          continue;
+        }
+        const int qb = nseg_q % C::QBUF;
+        const bool can_qk = have_q && (jq > 0 || mbar_test_wait(bars.q_full(qb), (nseg_q / C::QBUF) & 1)) &&
+                            mbar_test_wait(bars.k_full(gq % STAGES), (gq / STAGES) & 1) &&
+                            (gq == 0 || mbar_test_wait(C::P_SEP ? bars.s_free(t) : bars.o_done(t), (gq - 1) & 1));
+        if (can_qk) {
+          tc_fence_after();
+          tq = sbase + C::Q_OFF + (qb * NQ + t) * C::Q_TILE_BYTES;
+          issue_qk(gq % STAGES);
+          mma_commit(bars.s_full(t));
+          SD_TR(warp, gq, 0);
+          ++gq;
+          if (++jq == sq.ke - sq.kb) {
+            mma_commit(bars.q_empty(qb));  // this tile is done reading the segment's Q
+            have_q = next_seg(uq, u1, nkv, sq);
+            jq = 0;
+            ++nseg_q;
           }
-          if (SD_MMA_IDLE_NS > 0) __nanosleep(SD_MMA_IDLE_NS);  // idle poll: leave issue slots to the softmax
-          if ((++spins & 31u) == 0) {
-            if (*abort_flag) ok = false;
-            else if (clock64() - t_idle > kWaitLimitCycles) {
-              *abort_flag = 1;
-              atomicOr(err, sd::kDevErrTimeout);
-              ok = false;
-            }
+          t_idle = clock64();
+          continue;
+        }
+        if (SD_MMA_IDLE_NS > 0) __nanosleep(SD_MMA_IDLE_NS);  // idle poll: leave issue slots to the softmax
+        if ((++spins & 31u) == 0) {
+          if (*abort_flag) ok = false;
+          else if (clock64() - t_idle > kWaitLimitCycles) {
+            *abort_flag = 1;
+            atomicOr(err, sd::kDevErrTimeout);
+            ok = false;
           }
         }
-        gb += n;
-        ++nseg;
       }
       // Drain: all tensor-core work issued by this thread completes before TMEM is released.
       const uint32_t fin = bars.fin() + 8 * t;
@@ -433,6 +495,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
+  SD_SPAN(1);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);
@@ -454,6 +517,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     long long u = u0;
     Seg sg;
     int gi = 0;  // CTA-wide K/V tile count: the phase of every per-tile barrier
+    int nseg_done = 0;
     while (ok && next_seg(u, u1, nkv, sg)) {
     const int bh = sg.it / qpairs, q0 = (sg.it % qpairs) * (BM * NQ);
     float m_run = -INFINITY, l_run = 0.f;
@@ -524,6 +588,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // unit, or the FMA-pipe polynomial for POLY_PAIRS of every 8 pairs), then all packing, so
       // that a warp keeps many independent exp2 in flight instead of waiting on each pair.
       constexpr int EB = SD_EXP_BLOCK;
+      // Tuning switch: the special-function-unit exponentials on bf16 pairs (argument rounded to
+      // bf16 first). Only where the row sum comes out of P V, which then sums the same bf16 P.
+      constexpr bool kExpBf16 = SD_EXP_BF16 && C::L_IN_V;
 #pragma unroll
       for (int b = 0; b < BN / 2; b += EB) {
         float x[2 * EB];
@@ -534,15 +601,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int i = 0; i < EB; ++i) {
           if (((b + i) & 7) < C::POLY_PAIRS) {
             exp2_poly2(x[2 * i], x[2 * i + 1], x[2 * i], x[2 * i + 1]);
-          } else {
+          } else if (!kExpBf16) {
             x[2 * i] = ex2_approx(x[2 * i]);
             x[2 * i + 1] = ex2_approx(x[2 * i + 1]);
           }
         }
 #pragma unroll
         for (int i = 0; i < EB; ++i) {
-          if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x[2 * i], x[2 * i + 1]);
-          pk[b + i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+          if (kExpBf16 && ((b + i) & 7) >= C::POLY_PAIRS) {
+            pk[b + i] = ex2_bf16x2(pack_bf16x2(x[2 * i], x[2 * i + 1]));
+          } else {
+            if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x[2 * i], x[2 * i + 1]);
+            pk[b + i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+          }
         }
       }
       if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
@@ -584,6 +655,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_arrive(bars.p_full(t));
       if (tr) SD_TR(trole, gi, 6);
     }
+    if (tr && warp == C::SOFT_WARP0 && sg.ke < nkv && sg.kb == 0) SD_SEG(5);
     if (!ok || !__all_sync(0xffffffffu, wait_bar(bars.o_done(t), (gi - 1) & 1, abort_flag, err))) {
       ok = false;
       break;
@@ -609,32 +681,58 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int i = 0; i < C::NPV / 4; ++i) dst[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
       float2* ml = reinterpret_cast<float2*>(slot + NQ * BM * C::NPV) + slot_row;
       *ml = make_float2(m_run, lsum);
-      __threadfence();
-      atomicAdd(flags + blockIdx.x - 1, 1u);
+      // Publish: every softmax thread arrives on slot_written (release, CTA scope); one leader
+      // thread -- in the last softmax warp, usually the last to get here -- waits for all of them,
+      // then makes the slot visible device-wide with one fence and one flag increment.
+      mbar_arrive(bars.slot_written());
+      if (warp == C::SOFT_WARP0 + 4 * NQ - 1) {
+        if (!__all_sync(0xffffffffu, wait_bar(bars.slot_written(), 0, abort_flag, err))) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          __threadfence();
+          atomicAdd(flags + blockIdx.x - 1, 1u);
+        }
+        __syncwarp();
+      }
+      if (tr && warp == C::SOFT_WARP0) SD_SEG(1 + nseg_done);
+      ++nseg_done;
       continue;
     }
     if (sg.ke < nkv) {
       // Head piece: wait for the tail (the next CTA processed it at the start of its range), merge.
+      // One leader thread polls the flag, fences, resets the flag for the next launch and opens
+      // slot_ready (acquire/release at CTA scope) for the other softmax threads.
       float* slot = ws + static_cast<size_t>(blockIdx.x) * C::SLOT_FLOATS;
-      volatile unsigned int* f = flags + blockIdx.x;
-      const long long w0 = clock64();
-      bool got = true;
-      for (uint32_t it = 0; *f < static_cast<unsigned>(NQ * BM); ++it) {
-        __nanosleep(64);
-        if ((it & 63u) == 63u && (*abort_flag || clock64() - w0 > kWaitLimitCycles)) {
-          if (!*abort_flag) {
-            *abort_flag = 1;
-            atomicOr(err, sd::kDevErrTimeout);
+      if (tr && warp == C::SOFT_WARP0) SD_SEG(6);
+      if (warp == C::SOFT_WARP0 && lane == 0) {
+        volatile unsigned int* f = flags + blockIdx.x;
+        const long long w0 = clock64();
+        bool got = true;
+        for (uint32_t it = 0; *f == 0u; ++it) {
+          __nanosleep(64);
+          if ((it & 63u) == 63u && (*abort_flag || clock64() - w0 > kWaitLimitCycles)) {
+            if (!*abort_flag) {
+              *abort_flag = 1;
+              atomicOr(err, sd::kDevErrTimeout);
+            }
+            got = false;
+            break;
           }
-          got = false;
-          break;
+        }
+        if (got) {
+          __threadfence();
+          *f = 0u;
+          mbar_arrive(bars.slot_ready());
         }
       }
-      if (!got) {
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, wait_bar(bars.slot_ready(), 0, abort_flag, err))) {
         ok = false;
         break;
       }
-      __threadfence();
+      if (tr && warp == C::SOFT_WARP0) SD_SEG(7);
       const float4* src = reinterpret_cast<const float4*>(slot + static_cast<size_t>(slot_row) * C::NPV);
       const float2 ml = reinterpret_cast<const float2*>(slot + NQ * BM * C::NPV)[slot_row];
       const float m_all = fmaxf(m_run, ml.x);
@@ -648,9 +746,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         ov[4 * i + 3] = ov[4 * i + 3] * a_h + o4.w * a_t;
       }
       lsum = C::L_IN_V ? ov[C::DH] : lsum * a_h + ml.y * a_t;
-      // consumed: the last of the 2 * NQ * 128 arrivals (tail writers, then these readers) resets
-      // the flag for the next launch
-      if (atomicAdd(flags + blockIdx.x, 1u) == static_cast<unsigned>(2 * NQ * BM - 1)) atomicExch(flags + blockIdx.x, 0u);
     }
     const int qrow = q0 + t * BM + row;
     const float inv_l = 1.0f / lsum;
@@ -665,6 +760,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (i < n16) dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
     }
     if (tr) SD_TR(trole, gi - 1, 7);  // segment epilogue done
+    if (tr && warp == C::SOFT_WARP0) SD_SEG(1 + nseg_done);
+    ++nseg_done;
     }
   }
   tc_fence_before();
@@ -745,6 +842,20 @@ sd_status workspace(size_t bytes, cudaStream_t s, void** out) {
   *out = w.ptr;
   return SD_OK;
 }
+
+}  // namespace
+
+sd_status sd::attention_clear_handoff(cudaStream_t s) {
+  int dev = 0;
+  sd_status st = sd::cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st != SD_OK || dev >= 64) return st;
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  const Workspace& w = g_ws[dev];
+  if (!w.ptr) return SD_OK;
+  return sd::cuda_check(cudaMemsetAsync(w.ptr, 0, w.bytes, s), "cudaMemsetAsync(attention workspace)");
+}
+
+namespace {
 
 // Fixed scratch of sd_attention_noalloc: a file-scope device array, so that entry point never
 // allocates. Every device that loads the library holds it until the process exits. Zero at module
@@ -827,10 +938,19 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
     flags = reinterpret_cast<unsigned int*>(static_cast<char*>(p) + fbytes);
   }
   const float scale_log2 = scale * 1.4426950408889634f;
-  kern<<<static_cast<unsigned>(G), C::THREADS, C::SMEM_BYTES, s>>>(
-      mq, mk, mv, static_cast<__nv_bfloat16*>(o), static_cast<int>(Lq), static_cast<int>(Lk), static_cast<int>(dh),
-      scale_log2, err, g_debug_flags, static_cast<int>(qpairs), static_cast<int>(items), ws, flags);
-  return sd::cuda_check(cudaGetLastError(), "sd_attention launch");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(G));
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  cfg.attrs = attr;
+  cfg.numAttrs = sd::pdl_attr(&attr[0]);
+  return sd::cuda_check(
+      cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, static_cast<__nv_bfloat16*>(o), static_cast<int>(Lq),
+                         static_cast<int>(Lk), static_cast<int>(dh), scale_log2, err, g_debug_flags,
+                         static_cast<int>(qpairs), static_cast<int>(items), ws, flags),
+      "sd_attention launch");
 }
 
 }  // namespace
@@ -895,5 +1015,23 @@ extern "C" void sd_debug_set_fault(int flags) { g_debug_flags = flags; }
 extern "C" int sd_debug_trace(void* host, int64_t bytes) {
   if (bytes < static_cast<int64_t>(sizeof(g_trace))) return -1;
   return cudaMemcpyFromSymbol(host, g_trace, sizeof(g_trace)) == cudaSuccess ? 0 : -2;
+}
+extern "C" int sd_debug_span(void* host, int64_t bytes) {
+  if (bytes < static_cast<int64_t>(sizeof(g_span))) return -1;
+  return cudaMemcpyFromSymbol(host, g_span, sizeof(g_span)) == cudaSuccess ? 0 : -2;
+}
+extern "C" int sd_debug_seg(void* host, int64_t bytes) {
+  if (bytes < static_cast<int64_t>(sizeof(g_seg))) return -1;
+  return cudaMemcpyFromSymbol(host, g_seg, sizeof(g_seg)) == cudaSuccess ? 0 : -2;
+}
+extern "C" int sd_debug_span_smid(void* host, int64_t bytes) {
+  if (bytes < static_cast<int64_t>(sizeof(g_span_smid))) return -1;
+  return cudaMemcpyFromSymbol(host, g_span_smid, sizeof(g_span_smid)) == cudaSuccess ? 0 : -2;
+}
+extern "C" int sd_debug_span_seq(void* host, int64_t bytes) {  // and resets the launch counter
+  if (bytes < static_cast<int64_t>(sizeof(g_span_seq))) return -1;
+  if (cudaMemcpyFromSymbol(host, g_span_seq, sizeof(g_span_seq)) != cudaSuccess) return -2;
+  const unsigned int zero = 0;
+  return cudaMemcpyToSymbol(g_span_entries, &zero, sizeof(zero)) == cudaSuccess ? 0 : -3;
 }
 #endif

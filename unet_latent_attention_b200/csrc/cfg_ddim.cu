@@ -35,6 +35,8 @@ __device__ __forceinline__ float guided_step(float x, float eu, float ec, float 
 __global__ void __launch_bounds__(kThreads) cfg_ddim_vec4(const float4* x, const float4* __restrict__ eu,
                                                           const float4* __restrict__ ec, float4* xo,
                                                           int64_t n4, float w, float A, float Bc) {
+  sd::grid_dep_wait();
+  sd::grid_dep_launch();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n4; i += stride) {
     const float4 a = ld_stream(x + i), u = ld_stream(eu + i), c = ld_stream(ec + i);
@@ -51,6 +53,8 @@ __global__ void __launch_bounds__(kThreads) cfg_ddim_vec4(const float4* x, const
 __global__ void __launch_bounds__(kThreads) cfg_ddim_scalar(const float* x, const float* __restrict__ eu,
                                                             const float* __restrict__ ec, float* xo,
                                                             int64_t n, float w, float A, float Bc) {
+  sd::grid_dep_wait();
+  sd::grid_dep_launch();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * kThreads;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n; i += stride)
     xo[i] = guided_step(x[i], eu[i], ec[i], w, A, Bc);
@@ -61,6 +65,19 @@ int grid_for(int64_t items) {
   int64_t g = (items + kThreads - 1) / kThreads;
   if (g > cap) g = cap;
   return static_cast<int>(g < 1 ? 1 : g);
+}
+
+// Launch with programmatic stream serialization (see sd_internal.h).
+template <class... P, class... A>
+cudaError_t launch(int grid, cudaStream_t s, void (*kern)(P...), A... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  cfg.attrs = attr;
+  cfg.numAttrs = sd::pdl_attr(&attr[0]);
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<P>(args)...);
 }
 
 }  // namespace
@@ -87,17 +104,17 @@ extern "C" sd_status sd_cfg_ddim_step(const float* x, const float* eps_u, const 
   int64_t done = 0;
   if (vec && n >= 4) {
     const int64_t n4 = n / 4;
-    cfg_ddim_vec4<<<grid_for(n4), kThreads, 0, s>>>(reinterpret_cast<const float4*>(x),
-                                                     reinterpret_cast<const float4*>(eps_u),
-                                                     reinterpret_cast<const float4*>(eps_c),
-                                                     reinterpret_cast<float4*>(x_out), n4, w,
-                                                     static_cast<float>(A), static_cast<float>(Bc));
+    cudaError_t e = launch(grid_for(n4), s, cfg_ddim_vec4, reinterpret_cast<const float4*>(x),
+                           reinterpret_cast<const float4*>(eps_u), reinterpret_cast<const float4*>(eps_c),
+                           reinterpret_cast<float4*>(x_out), n4, w, static_cast<float>(A), static_cast<float>(Bc));
+    if (e != cudaSuccess) return sd::cuda_check(e, "sd_cfg_ddim_step launch");
     done = n4 * 4;
   }
   if (done < n) {
     const int64_t rest = n - done;
-    cfg_ddim_scalar<<<grid_for(rest), kThreads, 0, s>>>(x + done, eps_u + done, eps_c + done, x_out + done, rest,
-                                                         w, static_cast<float>(A), static_cast<float>(Bc));
+    return sd::cuda_check(launch(grid_for(rest), s, cfg_ddim_scalar, x + done, eps_u + done, eps_c + done,
+                                 x_out + done, rest, w, static_cast<float>(A), static_cast<float>(Bc)),
+                          "sd_cfg_ddim_step launch");
   }
-  return sd::cuda_check(cudaGetLastError(), "sd_cfg_ddim_step launch");
+  return SD_OK;
 }

@@ -119,6 +119,8 @@ __global__ void __launch_bounds__(THREADS) gn_resident(const float* x, const flo
   __shared__ Stats s_warp[THREADS / 32];
   __shared__ Stats s_all[kMaxCluster];
   __shared__ float s_mean, s_rstd;
+  sd::grid_dep_wait();
+  sd::grid_dep_launch();
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
   const int64_t grp = blockIdx.x / cluster.num_blocks();  // b * groups + g
@@ -178,6 +180,8 @@ __global__ void __launch_bounds__(kThreads) gn_streaming(const float* x, const f
   __shared__ Stats s_warp[kThreads / 32];
   __shared__ Stats s_all[kMaxCluster];
   __shared__ float s_mean, s_rstd;
+  sd::grid_dep_wait();
+  sd::grid_dep_launch();
   cg::cluster_group cluster = cg::this_cluster();
   const int64_t rank = cluster.block_rank();
   const int64_t grp = blockIdx.x / cluster.num_blocks();
@@ -225,13 +229,13 @@ cudaError_t launch_resident(dim3 grid, int cs, cudaStream_t s, const float* x, c
   cfg.gridDim = grid;
   cfg.blockDim = dim3(THREADS);
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1 + sd::pdl_attr(&attr[1]);
   return cudaLaunchKernelEx(&cfg, gn_resident<ITEMS, THREADS>, x, gamma, beta, y, group_elems, chunk, hw, cpg, groups, eps);
 }
 
@@ -306,13 +310,13 @@ extern "C" sd_status sd_group_norm(const float* x, const float* gamma, const flo
     cfg.gridDim = dim3(static_cast<unsigned>(n_groups * c));
     cfg.blockDim = dim3(kThreads);
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = c;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 1 + sd::pdl_attr(&attr[1]);
     err = cudaLaunchKernelEx(&cfg, gn_streaming, x, gamma, beta, y, group_elems, chunk, hw,
                              static_cast<int>(cpg), static_cast<int>(groups), eps);
   }

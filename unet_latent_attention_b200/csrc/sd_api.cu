@@ -88,6 +88,8 @@ sd_status sd_device_status(void* stream, int reset) {
   if (st != SD_OK) return st;
   if (reset) {
     st = sd::cuda_check(cudaMemsetAsync(word, 0, sizeof(unsigned int), s), "cudaMemsetAsync(status)");
+    // An aborted attention launch may have left hand-off flags set: clear them with the word.
+    if (st == SD_OK && host != 0) st = sd::attention_clear_handoff(s);
     if (st == SD_OK) st = sd::cuda_check(cudaStreamSynchronize(s), "cudaStreamSynchronize");
     if (st != SD_OK) return st;
   }

@@ -32,4 +32,34 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // Streaming-multiprocessor count of the current device (cached per device).
 int sm_count();
 
+// Clears the attention hand-off workspace of the current device on `s` (after a kernel gave up a
+// bounded wait, its flags may be left set).
+sd_status attention_clear_handoff(cudaStream_t s);
+
+// Programmatic dependent launch. Every kernel of the library is launched so that its CTAs may start
+// while the kernel before it on the stream is still finishing. Each kernel executes grid_dep_wait()
+// before its first global-memory access: that returns once the previous kernel has completed and its
+// memory operations are visible, so stream order is kept for all data. grid_dep_launch() lets the
+// next kernel on the stream start its own launch early. Both are no-ops when the launch carries no
+// programmatic dependency.
+#ifndef SD_PDL
+#define SD_PDL 1
+#endif
+#ifdef __CUDACC__
+__device__ __forceinline__ void grid_dep_wait() {
+  if (SD_PDL) asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  if (SD_PDL) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+#endif
+// Writes the programmatic-serialization launch attribute into `attr` (if enabled) and returns the
+// number of attributes written.
+inline unsigned int pdl_attr(cudaLaunchAttribute* attr) {
+  if (!SD_PDL) return 0;
+  attr->id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr->val.programmaticStreamSerializationAllowed = 1;
+  return 1;
+}
+
 }  // namespace sd
