@@ -106,6 +106,10 @@ constexpr int kTraceLast = 0;
 #define SD_EXP_BF16 0  // tuning: exp2 of bf16 pairs on the special-function unit (see the exp loop)
 #endif
 
+#ifndef SD_PING_RELEASE
+#define SD_PING_RELEASE -1  // tuning override of Cfg::PING_RELEASE (-1: the per-config choice)
+#endif
+
 #ifndef SD_PINGPONG
 #define SD_PINGPONG 1  // alternate the two query tiles' exp2 phases on each SM sub-partition
 #endif
@@ -188,6 +192,9 @@ struct Cfg {
   static_assert(NQ != 2 || 128 * REG_HELPER + 256 * REG_SOFT <= 168 * 384, "register split exceeds the launch budget");
   // Split-item hand-off slot: raw O (NPV fp32 per row) and (m, l) per row of the NQ tiles.
   static constexpr int SLOT_FLOATS = NQ * BM * (NPV + 2);
+  // Column pairs after which a softmax warp passes the ping-pong token (measured: half-way for
+  // dh 64, whose exp2 loop also sums the row in fp32; at the end of the loop otherwise).
+  static constexpr int PING_RELEASE = (DH == 64 && BN == 128) ? BN / 4 : BN / 2;
   // Of every 8 column pairs, this many take the FMA-pipe exp2 instead of the special-function unit.
   static constexpr int POLY_PAIRS = SD_POLY_PAIRS >= 0 ? SD_POLY_PAIRS : POLY_;
   static_assert(NPV % 16 == 0 && NPV <= 256, "MMA N must be a multiple of 16 and at most 256");
@@ -588,11 +595,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // unit, or the FMA-pipe polynomial for POLY_PAIRS of every 8 pairs), then all packing, so
       // that a warp keeps many independent exp2 in flight instead of waiting on each pair.
       constexpr int EB = SD_EXP_BLOCK;
+      // The token goes to the partner warp after kRelease column pairs: its exp2 phase then
+      // overlaps the rest of this one (two warps keep the special-function unit busier than one).
+      constexpr int kRel = SD_PING_RELEASE >= 0 ? SD_PING_RELEASE : C::PING_RELEASE;
+      constexpr int kRelease = kRel > BN / 2 ? BN / 2 : kRel / EB * EB;
       // Tuning switch: the special-function-unit exponentials on bf16 pairs (argument rounded to
       // bf16 first). Only where the row sum comes out of P V, which then sums the same bf16 P.
       constexpr bool kExpBf16 = SD_EXP_BF16 && C::L_IN_V;
 #pragma unroll
       for (int b = 0; b < BN / 2; b += EB) {
+        if (kPing && kRelease < BN / 2 && b == kRelease) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
+        }
         float x[2 * EB];
 #pragma unroll
         for (int i = 0; i < EB; ++i)  // s * scale * log2(e) - m, two columns per instruction
@@ -617,7 +632,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
       }
       if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
-      if (kPing) {
+      if (kPing && kRelease == BN / 2) {
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
       }
