@@ -106,6 +106,10 @@ constexpr int kTraceLast = 0;
 #define SD_EXP_BF16 0  // tuning: exp2 of bf16 pairs on the special-function unit (see the exp loop)
 #endif
 
+#ifndef SD_P_CHUNKED
+#define SD_P_CHUNKED -1  // tuning override of Cfg::CHUNK_P (-1: the per-config choice)
+#endif
+
 #ifndef SD_PING_RELEASE
 #define SD_PING_RELEASE -1  // tuning override of Cfg::PING_RELEASE (-1: the per-config choice)
 #endif
@@ -195,6 +199,9 @@ struct Cfg {
   // Column pairs after which a softmax warp passes the ping-pong token (measured: half-way for
   // dh 64, whose exp2 loop also sums the row in fp32; at the end of the loop otherwise).
   static constexpr int PING_RELEASE = (DH == 64 && BN == 128) ? BN / 4 : BN / 2;
+  // Store P in 16-column chunks inside the exp2 loop (measured: faster for the single short key
+  // tile of cross-attention, slower for the long key loops).
+  static constexpr bool CHUNK_P = BN < 128;
   // Of every 8 column pairs, this many take the FMA-pipe exp2 instead of the special-function unit.
   static constexpr int POLY_PAIRS = SD_POLY_PAIRS >= 0 ? SD_POLY_PAIRS : POLY_;
   static_assert(NPV % 16 == 0 && NPV <= 256, "MMA N must be a multiple of 16 and at most 256");
@@ -579,6 +586,31 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (tr) SD_TR(trole, gi, 3);
       const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
       if (rescale) m_run = m_new;
+      // With CHUNK_P, P goes to tensor memory in 16-column chunks as the exp2 loop produces it,
+      // which needs the previous P V complete (and O rescaled) first; waiting for it here does not
+      // hold the ping-pong token.
+      constexpr bool kChunkP = SD_P_CHUNKED >= 0 ? SD_P_CHUNKED != 0 : C::CHUNK_P;
+      if (kChunkP) {
+        if (C::P_SEP && gi > 0) {
+          if (!__all_sync(0xffffffffu, wait_bar(bars.o_done(t), (gi - 1) & 1, abort_flag, err))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        if (rescale && !first) {
+#pragma unroll
+          for (int c = 0; c < C::NPV / 16; ++c) {  // O columns, the row-sum column DH among them
+            const uint32_t addr = tO + c * 16;
+            uint32_t r[16];
+            tmem_ld16(addr, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st16(addr, r);
+          }
+        }
+      }
       // Ping-pong: the special-function unit of a sub-partition serves one tile's exp2 phase at a
       // time; the other tile's warp on it does its row max, P store and S load meanwhile. Tile 0
       // goes first; each warp hands the token to its partner (same sub-partition) after its exps.
@@ -630,6 +662,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             pk[b + i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
           }
         }
+        if (kChunkP && (b + EB) % 16 == 0) {  // 16 packed columns done: store them now
+          const int c = (b + EB) / 16 - 1;
+          uint32_t r[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) r[i] = pk[c * 16 + i];
+          tmem_st16(tP + c * 16, r);
+        }
       }
       if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
       if (kPing && kRelease == BN / 2) {
@@ -638,7 +677,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       if (tr) SD_TR(trole, gi, 4);
       // The previous P V (and the O it accumulates) must be complete before P and O are touched.
-      if (C::P_SEP && gi > 0) {
+      if (!kChunkP && C::P_SEP && gi > 0) {
         if (!__all_sync(0xffffffffu, wait_bar(bars.o_done(t), (gi - 1) & 1, abort_flag, err))) {
           ok = false;
           break;
@@ -646,7 +685,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tc_fence_after();
       }
       if (tr) SD_TR(trole, gi, 5);
-      if (rescale && !first) {
+      if (!kChunkP && rescale && !first) {
 #pragma unroll
         for (int c = 0; c < C::NPV / 16; ++c) {  // O columns, the row-sum column DH among them
           const uint32_t addr = tO + c * 16;
@@ -660,6 +699,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
+        if (kChunkP) break;
         uint32_t r[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) r[i] = pk[c * 16 + i];
