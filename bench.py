@@ -349,8 +349,9 @@ def _graph_time_us(fn, n, dev):
 
 def bench_extra(sdk, dev, hbm):
     """Labelled extras, not the headline: the 20-step guided DDIM loop of the batched-serving
-    workload (one CUDA graph), and a size sweep of GroupNorm and CFG+DDIM up to buffers far larger
-    than L2 that shows the asymptotic HBM bandwidth of these small-shape kernels."""
+    workload (one CUDA graph), a size sweep of GroupNorm and CFG+DDIM up to buffers far larger
+    than L2 that shows the asymptotic HBM bandwidth of these small-shape kernels, and
+    cross-attention with longer text contexts."""
     import torch
     out = {}
     lat = si.WORKLOADS[5].latent
@@ -383,6 +384,18 @@ def bench_extra(sdk, dev, hbm):
                       "frac_hbm": gbs / hbm})
         del a, u, c, o
     out["bandwidth_sweep"] = sweep
+    # Cross-attention at the SD1.5 512x512 top level with text contexts of 77, 256 and 512 tokens
+    # (24 rotating input sets, 126 MB of Q per pass: more than L2).
+    long = []
+    for Lk in (77, 256, 512):
+        sets = [(torch.randn(2, 8, 4096, 40, device=dev, dtype=torch.bfloat16),
+                 torch.randn(2, 8, Lk, 40, device=dev, dtype=torch.bfloat16),
+                 torch.randn(2, 8, Lk, 40, device=dev, dtype=torch.bfloat16)) for _ in range(24)]
+        outs = [torch.empty_like(s[0]) for s in sets]
+        us = _graph_time_us(lambda i: sdk.sd_attention(*sets[i % 24], out=outs[i % 24]), 24, dev)
+        long.append({"shape": [2, 8, 4096, Lk, 40], "us": us, "TFLOP/s": 4 * 2 * 8 * 4096 * Lk * 40 / (us * 1e-6) / 1e12})
+        del sets, outs
+    out["cross_attention_text_length"] = long
     torch.cuda.empty_cache()
     return out
 

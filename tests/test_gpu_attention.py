@@ -120,3 +120,17 @@ def test_repeated_launches_reuse_the_hand_off_flags(cuda):
         o = sdk.sd_attention(qd, kd, vd)
         sdk.sd_device_status()
         _check(o.float().cpu().numpy(), ref)
+
+
+LONG_TEXT = [si.AttnShape(2, 8, 4096, 256, 40), si.AttnShape(2, 8, 4096, 512, 40),
+             si.AttnShape(2, 10, 1024, 256, 64), si.AttnShape(2, 10, 1024, 512, 64)]
+
+
+@pytest.mark.parametrize("shape", LONG_TEXT, ids=[f"Lk{s.Lk}-dh{s.dh}" for s in LONG_TEXT])
+def test_long_text_cross_attention(cuda, shape):
+    # text contexts of 256 and 512 tokens (longer-text encoders): the key sequence spans 2-4 key
+    # tiles of the online softmax; sampled rows against the oracle
+    q, k, v = si.attention_qkv(6, shape, sub=shape.Lk + shape.dh)
+    o = _run(q, k, v, cuda)
+    rows = _sampled_rows(shape, 96, shape.Lk)
+    _check(o[rows[:, 0], rows[:, 1], rows[:, 2]], oracle.attention_rows(q, k, v, rows))
