@@ -376,6 +376,15 @@ def bench_extra(sdk, dev, hbm):
         sweep.append({"kernel": "group_norm", "shape": [B, C, H, W], "MB": 8 * B * C * H * W / 1e6, "us": us,
                       "GB/s": gbs, "frac_hbm": gbs / hbm})
         del xs, ys
+    for (B, C, H, W) in [(2, 320, 64, 64), (16, 640, 64, 64)]:  # GroupNorm + SiLU with a bf16 output
+        xs = [torch.randn(B, C, H, W, device=dev) for _ in range(2)]
+        gm, bt = torch.ones(C, device=dev), torch.zeros(C, device=dev)
+        ys = [torch.empty(B, C, H, W, device=dev, dtype=torch.bfloat16) for _ in range(2)]
+        us = _graph_time_us(lambda i: sdk.sd_group_norm_silu(xs[i % 2], gm, bt, 32, 1e-5, out=ys[i % 2]), 20, dev)
+        gbs = 6 * B * C * H * W / (us * 1e-6) / 1e9
+        sweep.append({"kernel": "group_norm_silu_bf16", "shape": [B, C, H, W], "MB": 6 * B * C * H * W / 1e6,
+                      "us": us, "GB/s": gbs, "frac_hbm": gbs / hbm})
+        del xs, ys
     for n in [1 << 20, 1 << 24, 1 << 26]:
         a, u, c, o = (torch.randn(n, device=dev) for _ in range(4))
         us = _graph_time_us(lambda i: sdk.sd_cfg_ddim_step(a, u, c, 7.5, 0.3, 0.5, out=o), 20, dev)

@@ -4,7 +4,7 @@
  * Three operations of one UNet denoising step, each an asynchronous launch on a caller stream:
  *
  *   sd_group_norm     GroupNorm of an NCHW fp32 activation (the reduction that feeds every UNet
- *                     block).
+ *                     block); sd_group_norm_silu fuses the SiLU that follows it.
  *   sd_attention      multi-head softmax(Q K^T * scale) V for the spatial-transformer blocks:
  *                     self-attention (K, V from the latent map, Lk = H*W) and cross-attention
  *                     (K, V from the projected 77-token text context).
@@ -66,6 +66,23 @@ sd_status sd_group_norm(const float* x, const float* gamma, const float* beta, f
                         void* stream);
 
 /*
+ * GroupNorm followed by SiLU in one launch: the GroupNorm + SiLU single-kernel fusion named in
+ * "从零实现扩散模型推理引擎：Rust + wgpu 的 GPU 加速图像生成架构" §9 (the activation that follows GroupNorm
+ * in the UNet's residual blocks). The page does not define SiLU; it is taken as
+ *   y = v * sigmoid(v) = v / (1 + exp(-v)),  v = GroupNorm(x) as in sd_group_norm.
+ *  x, gamma, beta, B..eps : as in sd_group_norm.
+ *  y        : [B, C, H, W] contiguous, fp32 (out_bf16 = 0) or bf16 (out_bf16 = 1, round to nearest
+ *             even), the input of the next convolution. With an fp32 output y may equal x (in
+ *             place); a bf16 y must not overlap x. Other overlaps: SD_ERR_INVALID_ARG.
+ *  out_bf16 : 0 or 1 (SD_ERR_INVALID_ARG otherwise).
+ * Same statistics, paths and errors as sd_group_norm; a bf16 y takes the single-read path when it
+ * is 8-byte aligned.
+ */
+sd_status sd_group_norm_silu(const float* x, const float* gamma, const float* beta, void* y,
+                             int64_t B, int64_t C, int64_t H, int64_t W, int64_t groups, float eps,
+                             int out_bf16, void* stream);
+
+/*
  * Attention, "从零实现扩散模型推理引擎：Rust + wgpu 的 GPU 加速图像生成架构" §3.2: for each batch b, head h
  * and query row i, O[b,h,i,:] = sum_j softmax_j(scale * Q[b,h,i,:] . K[b,h,j,:]) V[b,h,j,:].
  * The kernel is a flash-style forward pass (tiles of 128 queries x 128 keys, running max and
@@ -76,7 +93,7 @@ sd_status sd_group_norm(const float* x, const float* gamma, const float* beta, f
  *  o      : bf16 [B, heads, Lq, dh] contiguous; must not overlap q, k or v.
  *  dh     : one of 40, 64, 80, 160 (SD1.5 and SDXL head sizes); others are SD_ERR_UNSUPPORTED.
  *  scale  : finite; callers normally pass 1/sqrt(dh).
- *  Lq, Lk : >= 1, any value (ragged tails are masked). B*heads <= 65535.
+ *  Lq, Lk : >= 1 and <= 2^30, any value (ragged tails are masked). B*heads < 2^31.
  * All four pointers must be 16-byte aligned (SD_ERR_MISALIGNED otherwise).
  */
 sd_status sd_attention(const void* q, const void* k, const void* v, void* o,

@@ -4,6 +4,7 @@ Plain, slow, fp64 numpy restatements of what the CUDA library computes:
 
 * ``attention``       softmax(Q K^T * scale) V per (batch, head)             -> oracle/attention.py
 * ``group_norm``      per-group mean / biased variance, then per-channel affine -> oracle/group_norm.py
+* ``group_norm_silu`` SiLU (v * sigmoid(v)) of the GroupNorm output            -> oracle/group_norm.py
 * ``cfg_ddim_step``   classifier-free guidance followed by a deterministic DDIM update
                       (eta = 0), plus the scaled-linear noise schedule      -> oracle/ddim.py
 
@@ -22,10 +23,10 @@ pinned by ``tests/test_oracle_*.py`` against closed forms, invariants, hand-work
 independent library routines; none is "parity unpinned".
 """
 from .attention import attention, attention_rows, softmax_weights
-from .group_norm import group_norm, group_stats
+from .group_norm import group_norm, group_norm_silu, group_stats, silu
 from .ddim import (cfg, ddim_step, cfg_ddim_step, scaled_linear_betas, alphas_cumprod,
                    ddim_timesteps, ddim_schedule, cfg_ddim_loop)
 
-__all__ = ["attention", "attention_rows", "softmax_weights", "group_norm", "group_stats", "cfg",
-           "ddim_step", "cfg_ddim_step", "scaled_linear_betas", "alphas_cumprod", "ddim_timesteps",
+__all__ = ["attention", "attention_rows", "softmax_weights", "group_norm", "group_norm_silu", "group_stats",
+           "silu", "cfg", "ddim_step", "cfg_ddim_step", "scaled_linear_betas", "alphas_cumprod", "ddim_timesteps",
            "ddim_schedule", "cfg_ddim_loop"]

@@ -8,6 +8,10 @@ each channel c gets y = x_hat * gamma[c] + beta[c] (the standard GroupNorm affin
 
 The oracle computes the same statistics in the numerically safer two-pass form (mean first,
 then the mean of squared deviations), which equals the page's one-pass form in exact arithmetic.
+
+The engine page's §9 names GroupNorm + SiLU as one fused kernel without defining SiLU; it is taken
+as the sigmoid-weighted linear unit v * sigmoid(v) (the activation after GroupNorm in the UNet's
+residual blocks).
 """
 from __future__ import annotations
 
@@ -38,3 +42,16 @@ def group_norm(x, gamma, beta, groups: int = 32, eps: float = 1e-5) -> np.ndarra
     g = np.asarray(gamma, dtype=np.float64).reshape(bshape)
     b = np.asarray(beta, dtype=np.float64).reshape(bshape)
     return xhat * g + b
+
+
+def silu(v) -> np.ndarray:
+    """v * sigmoid(v) in fp64, written with exp(-|v|) so that no exponential overflows."""
+    v = np.asarray(v, dtype=np.float64)
+    e = np.exp(-np.abs(v))
+    sig = np.where(v >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+    return v * sig
+
+
+def group_norm_silu(x, gamma, beta, groups: int = 32, eps: float = 1e-5) -> np.ndarray:
+    """SiLU applied to the GroupNorm output (after the per-channel affine)."""
+    return silu(group_norm(x, gamma, beta, groups, eps))

@@ -53,6 +53,15 @@ def test_group_norm_argument_errors(L):
     assert L.sd_group_norm(0, 0, 0, 0, 0, 32, 4, 4, 32, 1e-5, None) == 0
 
 
+def test_group_norm_silu_argument_errors(L):
+    P = 1 << 12
+    assert L.sd_group_norm_silu(P, P, P, P + (1 << 20), 1, 32, 4, 4, 32, 1e-5, 2, None) == 1  # out_bf16 not 0/1
+    assert L.sd_group_norm_silu(P, P, P, P, 1, 32, 4, 4, 32, 1e-5, 1, None) == 1  # bf16 output in place
+    assert L.sd_group_norm_silu(P, P, P, P + 8, 1, 32, 4, 4, 32, 1e-5, 0, None) == 1  # partial overlap
+    assert L.sd_group_norm_silu(P, P, P, P, 1, 30, 4, 4, 32, 1e-5, 0, None) == 1  # 32 does not divide 30
+    assert L.sd_group_norm_silu(0, 0, 0, 0, 0, 32, 4, 4, 32, 1e-5, 1, None) == 0
+
+
 def test_cfg_ddim_argument_errors(L):
     P = 1 << 12
     assert L.sd_cfg_ddim_step(P, P + 4096, P + 8192, P, 16, 7.5, 0.0, 0.5, None) == 1  # alpha_t = 0

@@ -83,3 +83,56 @@ def test_large_mean_is_not_cancelled():
     _, v = oracle.group_stats(x, 2)
     _, v0 = oracle.group_stats(base, 2)
     np.testing.assert_allclose(v, 1e-4 * v0, rtol=1e-7)
+
+
+# ---- SiLU and the fused GroupNorm + SiLU (the engine page's §9 fusion; SiLU(v) = v * sigmoid(v))
+
+def test_silu_closed_forms():
+    # sigmoid(ln 3) = 3/4 and sigmoid(-ln 3) = 1/4
+    l3 = np.log(3.0)
+    np.testing.assert_allclose(oracle.silu(np.array([0.0, l3, -l3])), [0.0, 0.75 * l3, -0.25 * l3], rtol=1e-15,
+                               atol=0)
+
+
+def test_silu_odd_part_is_identity():
+    # v * s(v) - (-v) * s(-v) = v (s(v) + s(-v)) = v: catches a sign slip or sigmoid(-v) for sigmoid(v)
+    v = np.linspace(-50, 50, 2001)
+    np.testing.assert_allclose(oracle.silu(v) - oracle.silu(-v), v, rtol=0, atol=1e-12)
+
+
+def test_silu_minimum_is_minus_omega():
+    # min_v v*sigmoid(v) = -W(1/e) = -0.27846454276107380 (Lambert W), reached at v = -1 - W(1/e)
+    v = np.linspace(-1.2790, -1.2780, 20001)
+    y = oracle.silu(v)
+    assert abs(y.min() - (-0.27846454276107380)) < 1e-12
+    assert abs(v[y.argmin()] - (-1.27846454276107380)) < 1e-6
+
+
+def test_silu_tails_do_not_overflow():
+    y = oracle.silu(np.array([-1000.0, -40.0, 40.0, 1000.0]))
+    assert np.isfinite(y).all()
+    np.testing.assert_allclose(y, [0.0, -40.0 * np.exp(-40.0), 40.0, 1000.0], rtol=1e-14, atol=1e-300)
+
+
+def test_silu_against_torch_float64():
+    v = normal((4096,), 11).astype(np.float64) * 6
+    np.testing.assert_allclose(oracle.silu(v), torch.nn.functional.silu(torch.from_numpy(v)).numpy(), rtol=1e-14,
+                               atol=1e-15)
+
+
+def test_group_norm_silu_constant_group_gives_silu_of_beta():
+    # a constant group normalises to 0, so the output is SiLU(beta[c]): SiLU comes after the affine
+    x = np.full((1, 4, 3, 3), 2.5)
+    beta = np.array([-2.0, -0.5, 0.5, 3.0])
+    y = oracle.group_norm_silu(x, np.full(4, 7.0), beta, 2, 1e-5)
+    np.testing.assert_allclose(y, np.broadcast_to(oracle.silu(beta).reshape(1, 4, 1, 1), y.shape), rtol=1e-15)
+
+
+def test_group_norm_silu_against_torch_float64():
+    x = normal((2, 64, 6, 6), 12).astype(np.float64) * 3 + 1
+    gamma = 1 + 0.1 * normal((64,), 13).astype(np.float64)
+    beta = 0.1 * normal((64,), 14).astype(np.float64)
+    tx = torch.from_numpy(x)
+    ref = torch.nn.functional.silu(torch.nn.functional.group_norm(tx, 32, torch.from_numpy(gamma),
+                                                                  torch.from_numpy(beta), eps=1e-5)).numpy()
+    np.testing.assert_allclose(oracle.group_norm_silu(x, gamma, beta, 32, 1e-5), ref, atol=1e-12)

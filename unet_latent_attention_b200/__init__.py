@@ -5,6 +5,7 @@ Argument marshalling only: every step runs in the CUDA kernels behind the C ABI 
 CPU fallback: if the library is missing or the tensors are not on a CUDA device, the calls raise.
 
     sd_group_norm(x, gamma, beta, groups=32, eps=1e-5, out=None)
+    sd_group_norm_silu(x, gamma, beta, groups=32, eps=1e-5, out=None, out_dtype=None)
     sd_attention(q, k, v, scale=None, out=None)
     sd_cfg_ddim_step(x, eps_u, eps_c, w, alpha_t, alpha_prev, out=None)
     sd_cfg_ddim_step_from_noise_pred(x, noise_pred, w, alpha_t, alpha_prev, out=None)
@@ -47,13 +48,14 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         i64, f32, f64, vp, c_int = ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_void_p, ctypes.c_int
         L.sd_group_norm.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
+        L.sd_group_norm_silu.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, c_int, vp]
         L.sd_attention.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
         L.sd_attention_noalloc.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
         L.sd_cfg_ddim_step.argtypes = [vp, vp, vp, vp, i64, f32, f64, f64, vp]
         L.sd_device_status.argtypes = [vp, c_int]
         L.sd_debug_set_fault.argtypes = [c_int]
         L.sd_debug_set_fault.restype = None
-        for f in ("sd_group_norm", "sd_attention", "sd_attention_noalloc", "sd_cfg_ddim_step", "sd_device_status"):
+        for f in ("sd_group_norm", "sd_group_norm_silu", "sd_attention", "sd_attention_noalloc", "sd_cfg_ddim_step", "sd_device_status"):
             getattr(L, f).restype = c_int
         L.sd_status_string.argtypes = [c_int]
         L.sd_status_string.restype = ctypes.c_char_p
@@ -104,6 +106,28 @@ def sd_group_norm(x, gamma, beta, groups: int = 32, eps: float = 1e-5, out=None)
         raise ValueError("gamma/beta must have C elements and out the shape of x")
     _check("sd_group_norm", lib().sd_group_norm(x.data_ptr(), gamma.data_ptr(), beta.data_ptr(), out.data_ptr(),
                                                 B, C, H, W, groups, eps, _stream(x)))
+    return out
+
+
+def sd_group_norm_silu(x, gamma, beta, groups: int = 32, eps: float = 1e-5, out=None, out_dtype=None):
+    """SiLU(GroupNorm(x)) of fp32 NCHW ``x`` in one launch; the output is fp32 (``out`` may be ``x``)
+    or bf16 (``out_dtype=torch.bfloat16``)."""
+    import torch
+    if x.dtype != torch.float32 or gamma.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise ValueError("sd_group_norm_silu takes fp32 x, gamma, beta")
+    if x.dim() != 4:
+        raise ValueError("x must be [B, C, H, W]")
+    if out is None:
+        out = torch.empty(x.shape, dtype=out_dtype or torch.float32, device=x.device)
+    if out.dtype not in (torch.float32, torch.bfloat16) or out.shape != x.shape:
+        raise ValueError("out must be fp32 or bf16 with the shape of x")
+    _require_cuda(x, gamma, beta, out)
+    B, C, H, W = x.shape
+    if gamma.numel() != C or beta.numel() != C:
+        raise ValueError("gamma/beta must have C elements")
+    _check("sd_group_norm_silu", lib().sd_group_norm_silu(x.data_ptr(), gamma.data_ptr(), beta.data_ptr(),
+                                                          out.data_ptr(), B, C, H, W, groups, eps,
+                                                          1 if out.dtype == torch.bfloat16 else 0, _stream(x)))
     return out
 
 

@@ -13,12 +13,16 @@
 //    cancels when |mean| >> std. Every CTA of a cluster merges the per-CTA triples in rank order,
 //    so all of them obtain bit-identical statistics.
 //  * The tail is fused: y = x * a_c + b_c with a_c = rstd * gamma[c], b_c = beta[c] - mean * a_c.
+//    sd_group_norm_silu adds the SiLU activation, v * sigmoid(v), that follows GroupNorm in the
+//    UNet's residual blocks (the page's GroupNorm + SiLU single-kernel fusion, §9), with an fp32 or
+//    bf16 output.
 //
 // Shapes the resident path cannot hold (groups above 8 x 16384 elements, H*W not a multiple of 4,
 // pointers not 16-byte aligned) take the streaming path: the same cluster merge, but each CTA
 // sweeps its part twice (statistics, then normalise), so x is read twice (the second time mostly
 // from L2). Neither path uses global scratch memory.
 #include <cooperative_groups.h>
+#include <cuda_bf16.h>
 
 #include <cmath>
 
@@ -75,6 +79,34 @@ __device__ __forceinline__ void st_stream(float4* p, float4 v) {
                : "memory");
 }
 
+// Epilogues: the affine output in fp32 (sd_group_norm), or SiLU of it in fp32 or bf16.
+enum Epi : int { kAffine = 0, kSiluF32 = 1, kSiluBf16 = 2 };
+
+__device__ __forceinline__ float silu(float v) { return v / (1.0f + __expf(-v)); }
+
+// Stores four consecutive outputs (element index 4 * i4 of y).
+template <int EPI>
+__device__ __forceinline__ void store4(void* y, int64_t i4, float4 v) {
+  if constexpr (EPI != kAffine) v = make_float4(silu(v.x), silu(v.y), silu(v.z), silu(v.w));
+  if constexpr (EPI == kSiluBf16) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&lo);
+    u.y = *reinterpret_cast<const uint32_t*>(&hi);
+    asm volatile("st.global.cs.v2.b32 [%0], {%1,%2};" :: "l"(reinterpret_cast<uint2*>(y) + i4), "r"(u.x), "r"(u.y)
+                 : "memory");
+  } else {
+    st_stream(reinterpret_cast<float4*>(y) + i4, v);
+  }
+}
+
+template <int EPI>
+__device__ __forceinline__ void store1(void* y, int64_t i, float v) {
+  if constexpr (EPI != kAffine) v = silu(v);
+  if constexpr (EPI == kSiluBf16) reinterpret_cast<__nv_bfloat16*>(y)[i] = __float2bfloat16_rn(v);
+  else reinterpret_cast<float*>(y)[i] = v;
+}
+
 // Reduces the thread's triple over the CTA, pushes the CTA's triple into slot `rank` of every
 // cluster peer's shared memory, and after one cluster barrier merges the slots in rank order, so
 // that every CTA obtains the same mean and rstd (left in shared memory). No CTA touches another's
@@ -111,9 +143,9 @@ __device__ __forceinline__ void cluster_group_stats(Stats st, float eps, float* 
 
 // Resident path: one cluster of `cs` CTAs per (b, g); CTA `rank` owns elements
 // [rank*chunk, (rank+1)*chunk) of the group, chunk a multiple of 4, held in registers.
-template <int ITEMS, int THREADS>
+template <int ITEMS, int THREADS, int EPI>
 __global__ void __launch_bounds__(THREADS) gn_resident(const float* x, const float* __restrict__ gamma,
-                                                        const float* __restrict__ beta, float* y,
+                                                        const float* __restrict__ beta, void* y,
                                                         int group_elems, int chunk, int hw, int cpg, int groups,
                                                         float eps) {
   __shared__ Stats s_warp[THREADS / 32];
@@ -155,7 +187,7 @@ __global__ void __launch_bounds__(THREADS) gn_resident(const float* x, const flo
   cluster_group_stats(st, eps, &s_mean, &s_rstd, s_warp, s_all);
   const float mean = s_mean, rstd = s_rstd;
 
-  float4* yg = reinterpret_cast<float4*>(y + base);
+  const int64_t base4 = base >> 2;  // base is a multiple of 4 (chunk and group_elems are)
   const int e0 = rank * chunk;
 #pragma unroll
   for (int i = 0; i < ITEMS; ++i) {
@@ -164,8 +196,8 @@ __global__ void __launch_bounds__(THREADS) gn_resident(const float* x, const flo
       const int c = g * cpg + (e0 + idx * 4) / hw;  // hw % 4 == 0: a float4 never straddles channels
       const float a = rstd * __ldg(gamma + c);
       const float b = fmaf(-mean, a, __ldg(beta + c));
-      st_stream(yg + idx, make_float4(fmaf(v[i].x, a, b), fmaf(v[i].y, a, b), fmaf(v[i].z, a, b),
-                                      fmaf(v[i].w, a, b)));
+      store4<EPI>(y, base4 + idx, make_float4(fmaf(v[i].x, a, b), fmaf(v[i].y, a, b), fmaf(v[i].z, a, b),
+                                              fmaf(v[i].w, a, b)));
     }
   }
 }
@@ -173,8 +205,9 @@ __global__ void __launch_bounds__(THREADS) gn_resident(const float* x, const flo
 // Streaming path: any shape and alignment. CTA `rank` of the cluster owns elements [lo, hi) of the
 // group; sweep 1 builds the triple (exact stats of each run of four values, merged pairwise),
 // sweep 2 normalises.
+template <int EPI>
 __global__ void __launch_bounds__(kThreads) gn_streaming(const float* x, const float* __restrict__ gamma,
-                                                         const float* __restrict__ beta, float* y,
+                                                         const float* __restrict__ beta, void* y,
                                                          int64_t group_elems, int64_t chunk, int64_t hw, int cpg,
                                                          int groups, float eps) {
   __shared__ Stats s_warp[kThreads / 32];
@@ -189,7 +222,7 @@ __global__ void __launch_bounds__(kThreads) gn_streaming(const float* x, const f
   const int64_t lo = rank * chunk;
   const int64_t hi = lo + chunk < group_elems ? lo + chunk : group_elems;
   const float* xg = x + grp * group_elems;
-  float* yg = y + grp * group_elems;
+  const int64_t y0 = grp * group_elems;
 
   Stats st{0.f, 0.f, 0.f};
   for (int64_t e = lo + 4 * threadIdx.x; e < hi; e += 4 * kThreads) {
@@ -217,13 +250,13 @@ __global__ void __launch_bounds__(kThreads) gn_streaming(const float* x, const f
   for (int64_t e = lo + threadIdx.x; e < hi; e += kThreads) {
     const int c = g * cpg + static_cast<int>(e / hw);
     const float a = rstd * __ldg(gamma + c);
-    yg[e] = fmaf(xg[e], a, fmaf(-mean, a, __ldg(beta + c)));
+    store1<EPI>(y, y0 + e, fmaf(xg[e], a, fmaf(-mean, a, __ldg(beta + c))));
   }
 }
 
-template <int ITEMS, int THREADS>
+template <int ITEMS, int THREADS, int EPI>
 cudaError_t launch_resident(dim3 grid, int cs, cudaStream_t s, const float* x, const float* gamma,
-                            const float* beta, float* y, int group_elems, int chunk, int hw, int cpg, int groups,
+                            const float* beta, void* y, int group_elems, int chunk, int hw, int cpg, int groups,
                             float eps) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -236,37 +269,42 @@ cudaError_t launch_resident(dim3 grid, int cs, cudaStream_t s, const float* x, c
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1 + sd::pdl_attr(&attr[1]);
-  return cudaLaunchKernelEx(&cfg, gn_resident<ITEMS, THREADS>, x, gamma, beta, y, group_elems, chunk, hw, cpg, groups, eps);
+  return cudaLaunchKernelEx(&cfg, gn_resident<ITEMS, THREADS, EPI>, x, gamma, beta, y, group_elems, chunk, hw, cpg,
+                            groups, eps);
 }
 
-}  // namespace
-
-extern "C" sd_status sd_group_norm(const float* x, const float* gamma, const float* beta, float* y, int64_t B,
-                                   int64_t C, int64_t H, int64_t W, int64_t groups, float eps, void* stream) {
-  if (B < 0 || C < 0 || H < 0 || W < 0) return sd::fail(SD_ERR_INVALID_ARG, "sd_group_norm: negative size");
+// One GroupNorm launch with epilogue EPI; `name` prefixes error messages.
+template <int EPI>
+sd_status group_norm_impl(const char* name, const float* x, const float* gamma, const float* beta, void* y, int64_t B,
+                          int64_t C, int64_t H, int64_t W, int64_t groups, float eps, void* stream) {
+  if (B < 0 || C < 0 || H < 0 || W < 0) return sd::fail(SD_ERR_INVALID_ARG, "%s: negative size", name);
   if (groups <= 0 || (C > 0 && C % groups != 0))
-    return sd::fail(SD_ERR_INVALID_ARG, "sd_group_norm: groups must be positive and divide C");
-  if (!(eps > 0.f) || !std::isfinite(eps)) return sd::fail(SD_ERR_INVALID_ARG, "sd_group_norm: eps must be > 0");
+    return sd::fail(SD_ERR_INVALID_ARG, "%s: groups must be positive and divide C", name);
+  if (!(eps > 0.f) || !std::isfinite(eps)) return sd::fail(SD_ERR_INVALID_ARG, "%s: eps must be > 0", name);
   if (B == 0 || C == 0 || H == 0 || W == 0) return SD_OK;
-  if (!x || !gamma || !beta || !y) return sd::fail(SD_ERR_INVALID_ARG, "sd_group_norm: null pointer");
+  if (!x || !gamma || !beta || !y) return sd::fail(SD_ERR_INVALID_ARG, "%s: null pointer", name);
   const int64_t hw = H * W;
   const int64_t cpg = C / groups;
   const int64_t group_elems = cpg * hw;
   const int64_t n_groups = B * groups;
   if (group_elems > (int64_t(1) << 31) - 1 || n_groups * kMaxCluster > 0x7fffffff)
-    return sd::fail(SD_ERR_UNSUPPORTED, "sd_group_norm: tensor too large");
-  const int64_t bytes = B * C * hw * static_cast<int64_t>(sizeof(float));
+    return sd::fail(SD_ERR_UNSUPPORTED, "%s: tensor too large", name);
+  constexpr int64_t kOutBytes = EPI == kSiluBf16 ? 2 : 4;
+  const int64_t xbytes = B * C * hw * static_cast<int64_t>(sizeof(float)), ybytes = B * C * hw * kOutBytes;
   const int64_t pbytes = C * static_cast<int64_t>(sizeof(float));
-  if ((y != x && sd::overlaps(y, bytes, x, bytes)) || sd::overlaps(y, bytes, gamma, pbytes) ||
-      sd::overlaps(y, bytes, beta, pbytes))
-    return sd::fail(SD_ERR_INVALID_ARG, "sd_group_norm: y overlaps an input (only y == x is allowed)");
+  // In place (y == x) only with an fp32 output: each element is read before it is overwritten.
+  const bool in_place = EPI != kSiluBf16 && static_cast<const void*>(y) == static_cast<const void*>(x);
+  if ((!in_place && sd::overlaps(y, ybytes, x, xbytes)) || sd::overlaps(y, ybytes, gamma, pbytes) ||
+      sd::overlaps(y, ybytes, beta, pbytes))
+    return sd::fail(SD_ERR_INVALID_ARG, "%s: y overlaps an input (only y == x with an fp32 output is allowed)", name);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   // Resident path: a (cluster size, CTA size) pair that holds the group in registers (at most
   // kMaxItems float4 per thread, 8 for 1024-thread CTAs) with chunk a multiple of 4 elements.
   // Policy (measured on the SD shapes): the smallest cluster and CTA size that still put about
   // one CTA on every SM.
-  const bool vec_ok = hw % 4 == 0 && sd::aligned16(x) && sd::aligned16(y);
+  const bool y_vec = EPI == kSiluBf16 ? (reinterpret_cast<uintptr_t>(y) & 7u) == 0 : sd::aligned16(y);
+  const bool vec_ok = hw % 4 == 0 && sd::aligned16(x) && y_vec;
   int cs = 0, threads = 0;
   if (vec_ok) {
     const int64_t sms = sd::sm_count();
@@ -294,7 +332,7 @@ extern "C" sd_status sd_group_norm(const float* x, const float* gamma, const flo
     const int ge = static_cast<int>(group_elems), ihw = static_cast<int>(hw), icpg = static_cast<int>(cpg),
               ig = static_cast<int>(groups);
 #define SD_GN_CASE(N, T) \
-  if (threads == T && need <= N) err = launch_resident<N, T>(grid, cs, s, x, gamma, beta, y, ge, chunk, ihw, icpg, ig, eps); else
+  if (threads == T && need <= N) err = launch_resident<N, T, EPI>(grid, cs, s, x, gamma, beta, y, ge, chunk, ihw, icpg, ig, eps); else
 #define SD_GN_T(T) SD_GN_CASE(1, T) SD_GN_CASE(2, T) SD_GN_CASE(3, T) SD_GN_CASE(4, T) SD_GN_CASE(5, T) \
     SD_GN_CASE(6, T) SD_GN_CASE(8, T)
     SD_GN_T(256) SD_GN_T(512) SD_GN_T(1024) SD_GN_CASE(10, 256) SD_GN_CASE(12, 256) SD_GN_CASE(16, 256)
@@ -317,8 +355,23 @@ extern "C" sd_status sd_group_norm(const float* x, const float* gamma, const flo
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1 + sd::pdl_attr(&attr[1]);
-    err = cudaLaunchKernelEx(&cfg, gn_streaming, x, gamma, beta, y, group_elems, chunk, hw,
+    err = cudaLaunchKernelEx(&cfg, gn_streaming<EPI>, x, gamma, beta, y, group_elems, chunk, hw,
                              static_cast<int>(cpg), static_cast<int>(groups), eps);
   }
-  return sd::cuda_check(err, "sd_group_norm launch");
+  return sd::cuda_check(err, "group norm launch");
+}
+
+}  // namespace
+
+extern "C" sd_status sd_group_norm(const float* x, const float* gamma, const float* beta, float* y, int64_t B,
+                                   int64_t C, int64_t H, int64_t W, int64_t groups, float eps, void* stream) {
+  return group_norm_impl<kAffine>("sd_group_norm", x, gamma, beta, y, B, C, H, W, groups, eps, stream);
+}
+
+extern "C" sd_status sd_group_norm_silu(const float* x, const float* gamma, const float* beta, void* y, int64_t B,
+                                        int64_t C, int64_t H, int64_t W, int64_t groups, float eps, int out_bf16,
+                                        void* stream) {
+  if (out_bf16 != 0 && out_bf16 != 1) return sd::fail(SD_ERR_INVALID_ARG, "sd_group_norm_silu: out_bf16 must be 0 or 1");
+  return out_bf16 ? group_norm_impl<kSiluBf16>("sd_group_norm_silu", x, gamma, beta, y, B, C, H, W, groups, eps, stream)
+                  : group_norm_impl<kSiluF32>("sd_group_norm_silu", x, gamma, beta, y, B, C, H, W, groups, eps, stream);
 }
