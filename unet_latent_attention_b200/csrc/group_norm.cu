@@ -82,7 +82,10 @@ __device__ __forceinline__ void st_stream(float4* p, float4 v) {
 // Epilogues: the affine output in fp32 (sd_group_norm), or SiLU of it in fp32 or bf16.
 enum Epi : int { kAffine = 0, kSiluF32 = 1, kSiluBf16 = 2 };
 
-__device__ __forceinline__ float silu(float v) { return v / (1.0f + __expf(-v)); }
+// v * sigmoid(v). The division is the approximate one (reciprocal then multiply, 2 ulp): exact
+// IEEE division made the fused kernel compute-bound. For v < -88, 1 + exp(-v) is +inf and the
+// result is -0.
+__device__ __forceinline__ float silu(float v) { return __fdividef(v, 1.0f + __expf(-v)); }
 
 // Stores four consecutive outputs (element index 4 * i4 of y).
 template <int EPI>
