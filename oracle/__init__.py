@@ -7,6 +7,8 @@ Plain, slow, fp64 numpy restatements of what the CUDA library computes:
 * ``group_norm_silu`` SiLU (v * sigmoid(v)) of the GroupNorm output            -> oracle/group_norm.py
 * ``cfg_ddim_step``   classifier-free guidance followed by a deterministic DDIM update
                       (eta = 0), plus the scaled-linear noise schedule      -> oracle/ddim.py
+* ``cfg_dpmpp_2m_step`` guidance followed by a DPM-Solver++(2M) multistep update, plus
+                      Karras sigmas                                        -> oracle/dpmpp.py
 
 Sources, cited in each function by page title and section:
 
@@ -26,7 +28,10 @@ from .attention import attention, attention_rows, softmax_weights
 from .group_norm import group_norm, group_norm_silu, group_stats, silu
 from .ddim import (cfg, ddim_step, cfg_ddim_step, scaled_linear_betas, alphas_cumprod,
                    ddim_timesteps, ddim_schedule, cfg_ddim_loop)
+from .dpmpp import (lam, data_prediction, dpmpp_2m_step, cfg_dpmpp_2m_step, karras_sigmas, alpha_bar_of_sigma,
+                    sd_sigma_range, dpmpp_2m_schedule, cfg_dpmpp_2m_loop)
 
 __all__ = ["attention", "attention_rows", "softmax_weights", "group_norm", "group_norm_silu", "group_stats",
            "silu", "cfg", "ddim_step", "cfg_ddim_step", "scaled_linear_betas", "alphas_cumprod", "ddim_timesteps",
-           "ddim_schedule", "cfg_ddim_loop"]
+           "ddim_schedule", "cfg_ddim_loop", "lam", "data_prediction", "dpmpp_2m_step", "cfg_dpmpp_2m_step",
+           "karras_sigmas", "alpha_bar_of_sigma", "sd_sigma_range", "dpmpp_2m_schedule", "cfg_dpmpp_2m_loop"]
