@@ -350,8 +350,8 @@ def _graph_time_us(fn, n, dev):
 def bench_extra(sdk, dev, hbm):
     """Labelled extras, not the headline: the 20-step guided DDIM loop of the batched-serving
     workload (one CUDA graph), a size sweep of GroupNorm and CFG+DDIM up to buffers far larger
-    than L2 that shows the asymptotic HBM bandwidth of these small-shape kernels, and
-    cross-attention with longer text contexts."""
+    than L2 that shows the asymptotic HBM bandwidth of these small-shape kernels, the same loop with
+    DPM-Solver++(2M), and cross-attention with longer text contexts."""
     import torch
     out = {}
     lat = si.WORKLOADS[5].latent
@@ -366,6 +366,17 @@ def bench_extra(sdk, dev, hbm):
     n = int(np.prod(lat))
     out["cfg_ddim_20_steps_serving"] = {"shape": list(lat), "us_per_loop": us, "us_per_step": us / 20,
                                         "GB/s": 20 * 16 * n / (us * 1e-6) / 1e9}
+    # the same 20-step guided loop with DPM-Solver++(2M) on Karras sigmas (history buffer in place)
+    hist = torch.zeros(lat, device=dev)
+    dsched = sdk.dpmpp_2m_schedule(20)
+
+    def loop2(_):
+        for (a_p, a_t, a_n, order), (eu, ec) in zip(dsched, eps):
+            sdk.sd_cfg_dpmpp_2m_step(x, eu, ec, hist, 7.5, a_p, a_t, a_n, order, out=x, d_out=hist)
+    us = _graph_time_us(loop2, 5, dev)
+    byts = sum(24 if o == 2 else 20 for *_, o in dsched) * n
+    out["cfg_dpmpp_2m_20_steps_serving"] = {"shape": list(lat), "us_per_loop": us, "us_per_step": us / 20,
+                                            "GB/s": byts / (us * 1e-6) / 1e9}
     sweep = []
     for (B, C, H, W) in [(2, 320, 64, 64), (8, 320, 96, 96), (16, 640, 64, 64), (16, 320, 128, 128)]:
         xs = [torch.randn(B, C, H, W, device=dev) for _ in range(2)]
@@ -385,6 +396,14 @@ def bench_extra(sdk, dev, hbm):
         sweep.append({"kernel": "group_norm_silu_bf16", "shape": [B, C, H, W], "MB": 6 * B * C * H * W / 1e6,
                       "us": us, "GB/s": gbs, "frac_hbm": gbs / hbm})
         del xs, ys
+    for m in [1 << 24, 1 << 26]:  # DPM-Solver++(2M), order 2: 24 bytes per element
+        a, u, c, d, o, e = (torch.randn(m, device=dev) for _ in range(6))
+        us = _graph_time_us(lambda i: sdk.sd_cfg_dpmpp_2m_step(a, u, c, d, 7.5, 0.2, 0.3, 0.4, 2, out=o, d_out=e), 20,
+                            dev)
+        gbs = 24 * m / (us * 1e-6) / 1e9
+        sweep.append({"kernel": "cfg_dpmpp_2m", "elements": m, "MB": 24 * m / 1e6, "us": us, "GB/s": gbs,
+                      "frac_hbm": gbs / hbm})
+        del a, u, c, d, o, e
     for n in [1 << 20, 1 << 24, 1 << 26]:
         a, u, c, o = (torch.randn(n, device=dev) for _ in range(4))
         us = _graph_time_us(lambda i: sdk.sd_cfg_ddim_step(a, u, c, 7.5, 0.3, 0.5, out=o), 20, dev)

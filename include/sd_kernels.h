@@ -8,7 +8,8 @@
  *   sd_attention      multi-head softmax(Q K^T * scale) V for the spatial-transformer blocks:
  *                     self-attention (K, V from the latent map, Lk = H*W) and cross-attention
  *                     (K, V from the projected 77-token text context).
- *   sd_cfg_ddim_step  classifier-free guidance fused with a deterministic DDIM latent update.
+ *   sd_cfg_ddim_step  classifier-free guidance fused with a deterministic DDIM latent update;
+ *                     sd_cfg_dpmpp_2m_step fuses it with a DPM-Solver++(2M) update instead.
  *
  * Sources: "从零实现扩散模型推理引擎：Rust + wgpu 的 GPU 加速图像生成架构" (the Rust + wgpu engine page):
  * §1 sampling loop, §3.1 GroupNorm reduction, §3.2 flash cross-attention with online softmax, §4
@@ -142,6 +143,31 @@ sd_status sd_attention_noalloc(const void* q, const void* k, const void* v, void
  */
 sd_status sd_cfg_ddim_step(const float* x, const float* eps_u, const float* eps_c, float* x_out,
                            int64_t n, float w, double alpha_t, double alpha_prev, void* stream);
+
+/*
+ * Guided DPM-Solver++(2M) step. The engine page ("从零实现扩散模型推理引擎：Rust + wgpu 的 GPU 加速图像生成
+ * 架构" §4) keeps a DPM-Solver++ scheduler (order 1 = DDIM-equivalent, order 2 from a sample history,
+ * Karras sigmas, lower_order_final) without printing its update; this is the published
+ * DPM-Solver++(2M) multistep method (Lu et al. 2022) on cumulative products alpha_bar:
+ *   alpha = sqrt(alpha_bar), sigma = sqrt(1 - alpha_bar), lambda = log(alpha / sigma),
+ *   g = eps_u + w (eps_c - eps_u),  D = (x - sigma_t g) / alpha_t,  h = lambda_next - lambda_t,
+ *   order 1: x' = (sigma_next / sigma_t) x - alpha_next expm1(-h) D            (= the DDIM step)
+ *   order 2: r = (lambda_t - lambda_prev) / h,
+ *            x' = (sigma_next / sigma_t) x - alpha_next expm1(-h) ((1 + 1/(2r)) D - D_prev / (2r)).
+ * The step to alpha_next = 1 (sigma = 0, the end of sampling) must be order 1 and returns D.
+ *  x, eps_u, eps_c : fp32, n elements each (eps_* as in sd_cfg_ddim_step).
+ *  d_prev : fp32 n elements, the previous step's D (order 2 only; may be NULL for order 1).
+ *  x_out  : fp32 n, the new latent; may equal x.
+ *  d_out  : fp32 n, this step's D (the history for the next step); may equal d_prev.
+ *  alpha_t in (0, 1), alpha_next in (0, 1], alpha_prev in (0, 1) (order 2: distinct from alpha_t,
+ *  and alpha_next != alpha_t); order is 1 or 2. Other values, a NULL d_prev for order 2 and any
+ *  other overlap between outputs and inputs are SD_ERR_INVALID_ARG.
+ * All coefficients are formed in double on the host. Any alignment is accepted; 16-byte aligned
+ * pointers take the vectorised path.
+ */
+sd_status sd_cfg_dpmpp_2m_step(const float* x, const float* eps_u, const float* eps_c, const float* d_prev,
+                               float* x_out, float* d_out, int64_t n, float w, double alpha_prev,
+                               double alpha_t, double alpha_next, int order, void* stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* sd_status_string(sd_status status);

@@ -71,6 +71,28 @@ def test_cfg_ddim_argument_errors(L):
     assert L.sd_cfg_ddim_step(0, 0, 0, 0, 0, 7.5, 0.5, 0.6, None) == 0
 
 
+def test_dpmpp_argument_errors(L):
+    P, n = 1 << 12, 16
+    Q = [P + i * 4096 for i in range(6)]  # x, eu, ec, d_prev, x_out, d_out: disjoint
+    f = L.sd_cfg_dpmpp_2m_step
+    assert f(*Q, n, 7.5, 0.2, 0.3, 0.4, 3, None) == 1  # order must be 1 or 2
+    assert f(*Q, n, 7.5, 0.2, 1.0, 1.0, 1, None) == 1  # alpha_t = 1: sigma_t = 0
+    assert f(*Q, n, 7.5, 0.2, 0.3, 1.0, 2, None) == 1 and "first order" in _err(L)  # last step is order 1
+    assert f(*Q, n, 7.5, 0.3, 0.3, 0.4, 2, None) == 1  # alpha_prev = alpha_t
+    assert f(Q[0], Q[1], Q[2], 0, Q[4], Q[5], n, 7.5, 0.2, 0.3, 0.4, 2, None) == 1  # order 2 without history
+    assert f(Q[0], Q[1], Q[2], Q[3], Q[4], Q[0], n, 7.5, 0.2, 0.3, 0.4, 2, None) == 1  # d_out overlaps x
+    assert f(Q[0], Q[1], Q[2], Q[3], Q[3] + 4, Q[5], n, 7.5, 0.2, 0.3, 0.4, 2, None) == 1  # x_out over d_prev
+    assert f(0, 0, 0, 0, 0, 0, 0, 7.5, 0.2, 0.3, 0.4, 1, None) == 0  # empty
+
+
+def test_dpmpp_schedule_matches_the_oracle():
+    import oracle
+    ours, ref = sdk.dpmpp_2m_schedule(20), oracle.dpmpp_2m_schedule(20)
+    assert [o for *_, o in ours] == [o for *_, o in ref]
+    for a, b in zip(ours, ref):
+        assert max(abs(x - y) for x, y in zip(a[:3], b[:3])) < 1e-13
+
+
 def test_binding_refuses_cpu_tensors(L):
     q = torch.zeros(1, 1, 8, 40, dtype=torch.bfloat16)
     with pytest.raises(ValueError, match="CUDA"):

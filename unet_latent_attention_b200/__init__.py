@@ -9,6 +9,7 @@ CPU fallback: if the library is missing or the tensors are not on a CUDA device,
     sd_attention(q, k, v, scale=None, out=None)
     sd_cfg_ddim_step(x, eps_u, eps_c, w, alpha_t, alpha_prev, out=None)
     sd_cfg_ddim_step_from_noise_pred(x, noise_pred, w, alpha_t, alpha_prev, out=None)
+    sd_cfg_dpmpp_2m_step(x, eps_u, eps_c, d_prev, w, alpha_prev, alpha_t, alpha_next, order, out=None, d_out=None)
 """
 from __future__ import annotations
 
@@ -17,7 +18,7 @@ import math
 import os
 import re
 
-from .schedule import ddim_schedule, scaled_linear_alphas_cumprod  # noqa: F401  (host-side tables)
+from .schedule import ddim_schedule, dpmpp_2m_schedule, karras_alpha_bars, scaled_linear_alphas_cumprod  # noqa: F401
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsdk.so")
@@ -52,10 +53,12 @@ def lib() -> ctypes.CDLL:
         L.sd_attention.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
         L.sd_attention_noalloc.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
         L.sd_cfg_ddim_step.argtypes = [vp, vp, vp, vp, i64, f32, f64, f64, vp]
+        L.sd_cfg_dpmpp_2m_step.argtypes = [vp, vp, vp, vp, vp, vp, i64, f32, f64, f64, f64, c_int, vp]
         L.sd_device_status.argtypes = [vp, c_int]
         L.sd_debug_set_fault.argtypes = [c_int]
         L.sd_debug_set_fault.restype = None
-        for f in ("sd_group_norm", "sd_group_norm_silu", "sd_attention", "sd_attention_noalloc", "sd_cfg_ddim_step", "sd_device_status"):
+        for f in ("sd_group_norm", "sd_group_norm_silu", "sd_attention", "sd_attention_noalloc", "sd_cfg_ddim_step",
+                  "sd_cfg_dpmpp_2m_step", "sd_device_status"):
             getattr(L, f).restype = c_int
         L.sd_status_string.argtypes = [c_int]
         L.sd_status_string.restype = ctypes.c_char_p
@@ -195,6 +198,26 @@ def sd_cfg_ddim_step_from_noise_pred(x, noise_pred, w: float, alpha_t: float, al
     """Same step taking the UNet output for the batch [uncond, cond] (uncond half first)."""
     eps_u, eps_c = noise_pred.chunk(2, dim=0)
     return sd_cfg_ddim_step(x, eps_u, eps_c, w, alpha_t, alpha_prev, out=out)
+
+
+def sd_cfg_dpmpp_2m_step(x, eps_u, eps_c, d_prev, w: float, alpha_prev: float, alpha_t: float, alpha_next: float,
+                         order: int, out=None, d_out=None):
+    """Guided DPM-Solver++(2M) step; returns (x_next, d) where d is this step's data prediction (the
+    history for the next step). ``d_prev`` is the previous step's d (unused, may be None, for order 1);
+    ``out`` may be ``x`` and ``d_out`` may be ``d_prev``."""
+    import torch
+    for t in (x, eps_u, eps_c) + ((d_prev,) if d_prev is not None else ()):
+        if t.dtype != torch.float32 or t.shape != x.shape:
+            raise ValueError("sd_cfg_dpmpp_2m_step takes fp32 tensors of one shape")
+    if order == 2 and d_prev is None:
+        raise ValueError("order 2 needs d_prev")
+    out = torch.empty_like(x) if out is None else out
+    d_out = torch.empty_like(x) if d_out is None else d_out
+    _require_cuda(x, eps_u, eps_c, out, d_out, *((d_prev,) if d_prev is not None else ()))
+    _check("sd_cfg_dpmpp_2m_step", lib().sd_cfg_dpmpp_2m_step(
+        x.data_ptr(), eps_u.data_ptr(), eps_c.data_ptr(), d_prev.data_ptr() if d_prev is not None else None,
+        out.data_ptr(), d_out.data_ptr(), x.numel(), w, alpha_prev, alpha_t, alpha_next, int(order), _stream(x)))
+    return out, d_out
 
 
 def sd_device_status(stream=None, reset: bool = True) -> int:
