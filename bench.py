@@ -424,6 +424,16 @@ def bench_extra(sdk, dev, hbm):
         long.append({"shape": [2, 8, 4096, Lk, 40], "us": us, "TFLOP/s": 4 * 2 * 8 * 4096 * Lk * 40 / (us * 1e-6) / 1e12})
         del sets, outs
     out["cross_attention_text_length"] = long
+    # fp16 tensors (sd_attention_f16) on the SD1.5 512x512 self- and cross-attention shapes
+    f16 = []
+    for Lk in (4096, 77):
+        sets = [tuple(torch.randn(2, 8, L, 40, device=dev, dtype=torch.float16) for L in (4096, Lk, Lk))
+                for _ in range(12)]
+        outs = [torch.empty_like(s[0]) for s in sets]
+        us = _graph_time_us(lambda i: sdk.sd_attention(*sets[i % 12], out=outs[i % 12]), 12, dev)
+        f16.append({"shape": [2, 8, 4096, Lk, 40], "us": us, "TFLOP/s": 4 * 2 * 8 * 4096 * Lk * 40 / (us * 1e-6) / 1e12})
+        del sets, outs
+    out["attention_fp16"] = f16
     torch.cuda.empty_cache()
     return out
 

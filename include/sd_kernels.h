@@ -5,7 +5,8 @@
  *
  *   sd_group_norm     GroupNorm of an NCHW fp32 activation (the reduction that feeds every UNet
  *                     block); sd_group_norm_silu fuses the SiLU that follows it.
- *   sd_attention      multi-head softmax(Q K^T * scale) V for the spatial-transformer blocks:
+ *   sd_attention      multi-head softmax(Q K^T * scale) V for the spatial-transformer blocks
+ *                     (bf16; sd_attention_f16 takes fp16 tensors):
  *                     self-attention (K, V from the latent map, Lk = H*W) and cross-attention
  *                     (K, V from the projected 77-token text context).
  *   sd_cfg_ddim_step  classifier-free guidance fused with a deterministic DDIM latent update;
@@ -100,6 +101,17 @@ sd_status sd_group_norm_silu(const float* x, const float* gamma, const float* be
 sd_status sd_attention(const void* q, const void* k, const void* v, void* o,
                        int64_t B, int64_t heads, int64_t Lq, int64_t Lk, int64_t dh, float scale,
                        void* stream);
+
+/*
+ * sd_attention on IEEE fp16 tensors: the engine page's precision choice
+ * ("从零实现扩散模型推理引擎：Rust + wgpu 的 GPU 加速图像生成架构" §5.2, Precision::Fp16, named as enough
+ * for SD1.5/SDXL). q, k, v and o are fp16 [B, heads, L, dh]; everything else (arguments, layouts,
+ * alignment, errors, scratch) is as in sd_attention. The tensor cores multiply fp16 by fp16 with
+ * fp32 accumulation; P is rounded to fp16 for P V, and O is written as fp16 (round to nearest).
+ */
+sd_status sd_attention_f16(const void* q, const void* k, const void* v, void* o,
+                           int64_t B, int64_t heads, int64_t Lq, int64_t Lk, int64_t dh, float scale,
+                           void* stream);
 
 /*
  * sd_attention_noalloc -- the same computation, arguments, layouts and errors as sd_attention, for

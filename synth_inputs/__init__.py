@@ -58,6 +58,12 @@ def to_bf16_exact(a: np.ndarray):
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
 
 
+def to_f16_exact(a: np.ndarray):
+    """Round an fp32 array to IEEE fp16 (round-to-nearest-even) and return a torch fp16 tensor (CPU)."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.float16)
+
+
 # ---------------------------------------------------------------------------------------------
 # Workloads: Stable Diffusion UNet shapes. Attention tensors are [B, heads, L, dh]; GroupNorm
 # tensors are NCHW fp32; guidance/DDIM tensors are latents [n_img, 4, h, w] fp32.

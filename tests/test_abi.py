@@ -45,6 +45,14 @@ def test_attention_argument_errors(L):
     assert L.sd_attention(P, P, P, P, 1 << 31, 1, 8, 8, 40, 1.0, None) == 2
 
 
+def test_attention_f16_argument_errors(L):
+    P = 1 << 12
+    assert L.sd_attention_f16(P, P, P, P, 1, 1, 8, 8, 50, 1.0, None) == 2  # head dim
+    assert L.sd_attention_f16(P + 2, P, P, P, 1, 1, 8, 8, 40, 1.0, None) == 3  # misaligned
+    assert L.sd_attention_f16(P, P, P, P + 64, 1, 1, 8, 8, 40, 1.0, None) == 1  # o overlaps q
+    assert L.sd_attention_f16(0, 0, 0, 0, 0, 1, 8, 8, 40, 1.0, None) == 0
+
+
 def test_group_norm_argument_errors(L):
     P = 1 << 12
     assert L.sd_group_norm(P, P, P, P, 1, 30, 4, 4, 32, 1e-5, None) == 1  # 32 does not divide 30

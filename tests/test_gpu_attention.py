@@ -134,3 +134,44 @@ def test_long_text_cross_attention(cuda, shape):
     o = _run(q, k, v, cuda)
     rows = _sampled_rows(shape, 96, shape.Lk)
     _check(o[rows[:, 0], rows[:, 1], rows[:, 2]], oracle.attention_rows(q, k, v, rows))
+
+
+# ---- fp16 tensors (sd_attention_f16), same gate as bf16
+
+def _qkv16(B, H, Lq, Lk, dh, seed):
+    return (si.to_f16_exact(si.normal((B, H, Lq, dh), seed)), si.to_f16_exact(si.normal((B, H, Lk, dh), seed + 1)),
+            si.to_f16_exact(si.normal((B, H, Lk, dh), seed + 2)))
+
+
+@pytest.mark.parametrize("dh", [40, 64, 80, 160])
+@pytest.mark.parametrize("Lq,Lk", [(7, 77), (129, 255), (513, 640)])
+def test_fp16_small_shapes(cuda, dh, Lq, Lk):
+    q, k, v = _qkv16(2, 3, Lq, Lk, dh, 12000 + dh + Lq + Lk)
+    o = sdk.sd_attention(q.to(cuda), k.to(cuda), v.to(cuda))
+    sdk.sd_device_status()
+    assert o.dtype == torch.float16
+    _check(o.float().cpu().numpy(), oracle.attention(q, k, v))
+
+
+def test_fp16_single_key_returns_v(cuda):
+    q, k, v = _qkv16(1, 2, 200, 1, 40, 12100)
+    o = sdk.sd_attention(q.to(cuda), k.to(cuda), v.to(cuda))
+    sdk.sd_device_status()
+    np.testing.assert_array_equal(o.float().cpu().numpy(), np.broadcast_to(v.float().numpy(), o.shape))
+
+
+@pytest.mark.parametrize("dh,heads,Lq,Lk", [(40, 8, 4096, 4096), (64, 10, 1024, 1024), (40, 8, 4096, 77)])
+def test_fp16_sd_shapes(cuda, dh, heads, Lq, Lk):
+    # SD1.5 / SDXL self- and cross-attention shapes, sampled rows (split items included)
+    shape = si.AttnShape(2, heads, Lq, Lk, dh)
+    q, k, v = _qkv16(2, heads, Lq, Lk, dh, 12200 + dh + Lk)
+    o = sdk.sd_attention(q.to(cuda), k.to(cuda), v.to(cuda))
+    sdk.sd_device_status()
+    rows = _sampled_rows(shape, 96, 12300 + dh)
+    _check(o.float().cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]], oracle.attention_rows(q, k, v, rows))
+
+
+def test_mixed_types_are_refused(cuda):
+    q = torch.zeros(1, 1, 8, 40, dtype=torch.float16, device=cuda)
+    with pytest.raises(ValueError):
+        sdk.sd_attention(q, q.to(torch.bfloat16), q)

@@ -6,7 +6,7 @@ CPU fallback: if the library is missing or the tensors are not on a CUDA device,
 
     sd_group_norm(x, gamma, beta, groups=32, eps=1e-5, out=None)
     sd_group_norm_silu(x, gamma, beta, groups=32, eps=1e-5, out=None, out_dtype=None)
-    sd_attention(q, k, v, scale=None, out=None)
+    sd_attention(q, k, v, scale=None, out=None)          (bf16 or fp16)
     sd_cfg_ddim_step(x, eps_u, eps_c, w, alpha_t, alpha_prev, out=None)
     sd_cfg_ddim_step_from_noise_pred(x, noise_pred, w, alpha_t, alpha_prev, out=None)
     sd_cfg_dpmpp_2m_step(x, eps_u, eps_c, d_prev, w, alpha_prev, alpha_t, alpha_next, order, out=None, d_out=None)
@@ -52,12 +52,14 @@ def lib() -> ctypes.CDLL:
         L.sd_group_norm_silu.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, c_int, vp]
         L.sd_attention.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
         L.sd_attention_noalloc.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
+        L.sd_attention_f16.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
         L.sd_cfg_ddim_step.argtypes = [vp, vp, vp, vp, i64, f32, f64, f64, vp]
         L.sd_cfg_dpmpp_2m_step.argtypes = [vp, vp, vp, vp, vp, vp, i64, f32, f64, f64, f64, c_int, vp]
         L.sd_device_status.argtypes = [vp, c_int]
         L.sd_debug_set_fault.argtypes = [c_int]
         L.sd_debug_set_fault.restype = None
-        for f in ("sd_group_norm", "sd_group_norm_silu", "sd_attention", "sd_attention_noalloc", "sd_cfg_ddim_step",
+        for f in ("sd_group_norm", "sd_group_norm_silu", "sd_attention", "sd_attention_noalloc", "sd_attention_f16",
+                  "sd_cfg_ddim_step",
                   "sd_cfg_dpmpp_2m_step", "sd_device_status"):
             getattr(L, f).restype = c_int
         L.sd_status_string.argtypes = [c_int]
@@ -135,10 +137,11 @@ def sd_group_norm_silu(x, gamma, beta, groups: int = 32, eps: float = 1e-5, out=
 
 
 def sd_attention(q, k, v, scale: float | None = None, out=None):
-    """softmax(q k^T * scale) v for bf16 q [B,h,Lq,dh], k/v [B,h,Lk,dh]; scale defaults to 1/sqrt(dh)."""
+    """softmax(q k^T * scale) v for q [B,h,Lq,dh], k/v [B,h,Lk,dh], all bf16 or all fp16 (the output
+    has the same type); scale defaults to 1/sqrt(dh)."""
     import torch
-    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
-        raise ValueError("sd_attention takes bf16 q, k, v")
+    if q.dtype not in (torch.bfloat16, torch.float16) or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("sd_attention takes q, k, v all bf16 or all fp16")
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
         raise ValueError("q, k, v must be [B, heads, L, dh]")
     B, Hh, Lq, dh = q.shape
@@ -147,12 +150,13 @@ def sd_attention(q, k, v, scale: float | None = None, out=None):
     if out is None:
         out = torch.empty_like(q)
     _require_cuda(q, k, v, out)
-    if out.shape != q.shape or out.dtype != torch.bfloat16:
-        raise ValueError("out must be bf16 with the shape of q")
+    if out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must have the shape and type of q")
     if scale is None:
         scale = 1.0 / math.sqrt(dh)
-    _check("sd_attention", lib().sd_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hh, Lq,
-                                              k.shape[2], dh, scale, _stream(q)))
+    name = "sd_attention_f16" if q.dtype == torch.float16 else "sd_attention"
+    _check(name, getattr(lib(), name)(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hh, Lq,
+                                      k.shape[2], dh, scale, _stream(q)))
     return out
 
 

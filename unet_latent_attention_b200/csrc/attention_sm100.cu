@@ -149,8 +149,10 @@ constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at B200 clocks
 // L_IN_V: the softmax row sums come out of the P V product itself: a fix-up warp writes bf16 1.0
 //         into column DH of every V tile once it lands (the TMA zero-fills columns >= DH), so O's
 //         column DH accumulates sum_j P_ij with no extra MMA (else fp32 adds in registers).
-template <int DH_, int BN_, int NQ_, int STAGES_, bool P_SEP_, bool L_IN_V_, int POLY_ = 0>
+// F16: the tensors (and P) are fp16 instead of bf16.
+template <int DH_, int BN_, int NQ_, int STAGES_, bool P_SEP_, bool L_IN_V_, int POLY_ = 0, bool F16_ = false>
 struct Cfg {
+  static constexpr bool F16 = F16_;
   static constexpr int DH = DH_;          // true head dim
   static constexpr int DHP = (DH + 15) / 16 * 16;  // Q K^T depth padded to the MMA granule (16)
   static constexpr int BN = BN_;          // keys per K/V tile
@@ -271,7 +273,7 @@ __device__ __forceinline__ bool next_seg(long long& u, long long u1, int nkv, Se
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, __nv_bfloat16* __restrict__ out, int Lq, int Lk,
+                   const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out, int Lq, int Lk,
                    int dh, float scale_log2, unsigned int* err, int debug_flags, int qpairs, int items,
                    float* __restrict__ ws, unsigned int* flags) {
   constexpr int BN = C::BN, NQ = C::NQ, STAGES = C::STAGES, NCH = C::NCH, NCHV = C::NCHV, DHP = C::DHP;
@@ -396,8 +398,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // hundreds of cycles, so two tiles' instruction streams must not queue behind each other.
     const int t = warp - 1;
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, C::NPV, true);
+      constexpr uint32_t idesc_qk = idesc_f16kind_f32(BM, BN, false, C::F16);
+      constexpr uint32_t idesc_pv = idesc_f16kind_f32(BM, C::NPV, true, C::F16);
       uint32_t tq = sbase + C::Q_OFF + t * C::Q_TILE_BYTES;  // the current segment's Q buffer
       auto issue_qk = [&](int s) {  // S = Q K_s^T over the padded head dim
         const uint32_t d = tmem + t * C::TM_TILE + C::TM_S;
@@ -501,7 +503,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       uint8_t* vt = smem + C::V_OFF + s * C::V_TILE_BYTES + ch * BN * 128;
 #pragma unroll
       for (int r = lane; r < BN; r += 32)
-        *reinterpret_cast<uint16_t*>(vt + r * 128 + ((g ^ (r & 7)) << 4) + gb) = 0x3F80u;  // bf16 1.0
+        *reinterpret_cast<uint16_t*>(vt + r * 128 + ((g ^ (r & 7)) << 4) + gb) = C::F16 ? 0x3C00u : 0x3F80u;  // 1.0
       fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.v_ready(s));
@@ -633,7 +635,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       constexpr int kRelease = kRel > BN / 2 ? BN / 2 : kRel / EB * EB;
       // Tuning switch: the special-function-unit exponentials on bf16 pairs (argument rounded to
       // bf16 first). Only where the row sum comes out of P V, which then sums the same bf16 P.
-      constexpr bool kExpBf16 = SD_EXP_BF16 && C::L_IN_V;
+      constexpr bool kExpBf16 = SD_EXP_BF16 && C::L_IN_V && !C::F16;
 #pragma unroll
       for (int b = 0; b < BN / 2; b += EB) {
         if (kPing && kRelease < BN / 2 && b == kRelease) {
@@ -659,7 +661,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             pk[b + i] = ex2_bf16x2(pack_bf16x2(x[2 * i], x[2 * i + 1]));
           } else {
             if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x[2 * i], x[2 * i + 1]);
-            pk[b + i] = pack_bf16x2(x[2 * i], x[2 * i + 1]);
+            pk[b + i] = C::F16 ? pack_f16x2(x[2 * i], x[2 * i + 1]) : pack_bf16x2(x[2 * i], x[2 * i + 1]);
           }
         }
         if (kChunkP && (b + EB) % 16 == 0) {  // 16 packed columns done: store them now
@@ -806,7 +808,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const float inv_l = 1.0f / lsum;
     uint32_t packed[DHP / 2];
 #pragma unroll
-    for (int i = 0; i < DHP / 2; ++i) packed[i] = pack_bf16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l);
+    for (int i = 0; i < DHP / 2; ++i)
+      packed[i] = C::F16 ? pack_f16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l)
+                         : pack_bf16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l);
     if (qrow < Lq) {
       uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * Lq + qrow) * dh);
       const int n16 = dh / 8;  // 16-byte groups of 8 bf16
@@ -840,7 +844,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 3-D map over a contiguous bf16 [planes, rows, dh] tensor, box {64, box_rows, 1}, 128-byte swizzle.
-sd_status make_map(CUtensorMap* map, const void* ptr, int64_t dh, int64_t rows, int64_t planes, int box_rows) {
+sd_status make_map(CUtensorMap* map, const void* ptr, int64_t dh, int64_t rows, int64_t planes, int box_rows,
+                   bool f16) {
   auto fn = encode_fn();
   if (!fn) return sd::fail(SD_ERR_CUDA, "sd_attention: cuTensorMapEncodeTiled is unavailable");
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(dh), static_cast<cuuint64_t>(rows),
@@ -848,7 +853,8 @@ sd_status make_map(CUtensorMap* map, const void* ptr, int64_t dh, int64_t rows, 
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(dh * 2), static_cast<cuuint64_t>(rows * dh * 2)};
   const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+  const CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                        const_cast<void*>(ptr), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return sd::fail(SD_ERR_CUDA, "sd_attention: cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -945,9 +951,9 @@ template <class C>
 sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t BH, int64_t Lq, int64_t Lk,
                  int64_t dh, float scale, cudaStream_t s, bool fixed = false) {
   CUtensorMap mq, mk, mv;
-  sd_status st = make_map(&mq, q, dh, Lq, BH, BM);
-  if (st == SD_OK) st = make_map(&mk, k, dh, Lk, BH, C::BN);
-  if (st == SD_OK) st = make_map(&mv, v, dh, Lk, BH, C::BN);
+  sd_status st = make_map(&mq, q, dh, Lq, BH, BM, C::F16);
+  if (st == SD_OK) st = make_map(&mk, k, dh, Lk, BH, C::BN, C::F16);
+  if (st == SD_OK) st = make_map(&mv, v, dh, Lk, BH, C::BN, C::F16);
   if (st != SD_OK) return st;
   unsigned int* err = sd::device_status_word();
   if (!err) return SD_ERR_CUDA;
@@ -1002,7 +1008,7 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
   cfg.attrs = attr;
   cfg.numAttrs = sd::pdl_attr(&attr[0]);
   return sd::cuda_check(
-      cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, static_cast<__nv_bfloat16*>(o), static_cast<int>(Lq),
+      cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, static_cast<uint16_t*>(o), static_cast<int>(Lq),
                          static_cast<int>(Lk), static_cast<int>(dh), scale_log2, err, g_debug_flags,
                          static_cast<int>(qpairs), static_cast<int>(items), ws, flags),
       "sd_attention launch");
@@ -1012,8 +1018,28 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
 
 namespace {
 
+// The launch table: a configuration per head dim and key length, for one element type.
+template <bool F16>
+sd_status dispatch(const void* q, const void* k, const void* v, void* o, int64_t BH, int64_t Lq, int64_t Lk,
+                   int64_t dh, float scale, cudaStream_t s, bool fixed) {
+  if (Lk <= 96) {  // short key sequence (the 77-token text context): one 96-key tile, no online rescale
+    switch (dh) {
+      case 40: return launch<Cfg<40, 96, SD_CROSS_NQ, 2, true, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+      case 64: return launch<Cfg<64, 96, SD_CROSS_NQ, 2, true, false, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+      case 80: return launch<Cfg<80, 96, SD_CROSS_NQ, 2, true, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+      default: break;  // dh = 160 already uses 64-key tiles
+    }
+  }
+  switch (dh) {
+    case 40: return launch<Cfg<40, 128, 2, SD_STAGES_SMALL, true, true, 2, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+    case 64: return launch<Cfg<64, 128, 2, SD_STAGES_SMALL, true, false, 2, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+    case 80: return launch<Cfg<80, 128, 2, 2, false, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+    default: return launch<Cfg<160, 64, 1, 3, true, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+  }
+}
+
 sd_status attention_impl(const void* q, const void* k, const void* v, void* o, int64_t B, int64_t heads, int64_t Lq,
-                         int64_t Lk, int64_t dh, float scale, void* stream, bool fixed) {
+                         int64_t Lk, int64_t dh, float scale, void* stream, bool fixed, bool f16 = false) {
   if (B < 0 || heads < 0 || Lq < 0 || Lk < 0) return sd::fail(SD_ERR_INVALID_ARG, "sd_attention: negative size");
   if (dh != 40 && dh != 64 && dh != 80 && dh != 160)
     return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention: head dim %lld not in {40, 64, 80, 160}", (long long)dh);
@@ -1030,20 +1056,8 @@ sd_status attention_impl(const void* q, const void* k, const void* v, void* o, i
   if (sd::overlaps(o, qbytes, q, qbytes) || sd::overlaps(o, qbytes, k, kvbytes) || sd::overlaps(o, qbytes, v, kvbytes))
     return sd::fail(SD_ERR_INVALID_ARG, "sd_attention: o overlaps q, k or v");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (Lk <= 96) {  // short key sequence (the 77-token text context): one 96-key tile, no online rescale
-    switch (dh) {
-      case 40: return launch<Cfg<40, 96, SD_CROSS_NQ, 2, true, true, 0>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-      case 64: return launch<Cfg<64, 96, SD_CROSS_NQ, 2, true, false>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-      case 80: return launch<Cfg<80, 96, SD_CROSS_NQ, 2, true, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-      default: break;  // dh = 160 already uses 64-key tiles
-    }
-  }
-  switch (dh) {
-    case 40: return launch<Cfg<40, 128, 2, SD_STAGES_SMALL, true, true, 2>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-    case 64: return launch<Cfg<64, 128, 2, SD_STAGES_SMALL, true, false, 2>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-    case 80: return launch<Cfg<80, 128, 2, 2, false, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-    default: return launch<Cfg<160, 64, 1, 3, true, true>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-  }
+  return f16 ? dispatch<true>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed)
+             : dispatch<false>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
 }
 
 }  // namespace
@@ -1051,6 +1065,12 @@ sd_status attention_impl(const void* q, const void* k, const void* v, void* o, i
 extern "C" sd_status sd_attention(const void* q, const void* k, const void* v, void* o, int64_t B, int64_t heads,
                                   int64_t Lq, int64_t Lk, int64_t dh, float scale, void* stream) {
   return attention_impl(q, k, v, o, B, heads, Lq, Lk, dh, scale, stream, false);
+}
+
+// The same attention on fp16 tensors (see sd_kernels.h).
+extern "C" sd_status sd_attention_f16(const void* q, const void* k, const void* v, void* o, int64_t B, int64_t heads,
+                                      int64_t Lq, int64_t Lk, int64_t dh, float scale, void* stream) {
+  return attention_impl(q, k, v, o, B, heads, Lq, Lk, dh, scale, stream, false, true);
 }
 
 // Same computation for callers that cannot allocate device memory (see sd_kernels.h): scratch comes

@@ -160,14 +160,20 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D, M x N tile; b_mn_major selects
 // an N-contiguous (MN-major) B operand.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
-  return (1u << 4)                       // D format: f32
-         | (1u << 7)                     // A format: bf16
-         | (1u << 10)                    // B format: bf16
-         | (0u << 15)                    // A K-major
+// kind::f16 instruction descriptor with an f32 accumulator; A and B are both bf16 or both f16
+// (the two operands of one MMA always share the type).
+__host__ __device__ constexpr uint32_t idesc_f16kind_f32(int M, int N, bool b_mn_major, bool f16) {
+  return (1u << 4)                          // D format: f32
+         | ((f16 ? 0u : 1u) << 7)           // A format: f16 (0) or bf16 (1)
+         | ((f16 ? 0u : 1u) << 10)          // B format: the same
+         | (0u << 15)                       // A K-major
          | ((b_mn_major ? 1u : 0u) << 16)
          | (static_cast<uint32_t>(N >> 3) << 17)
          | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool b_mn_major) {
+  return idesc_f16kind_f32(M, N, b_mn_major, false);
 }
 
 // Make generic-proxy writes to shared memory visible to the async proxy (TMA, tensor core).
@@ -243,6 +249,12 @@ __device__ __forceinline__ uint32_t ex2_bf16x2(uint32_t x) {
   uint32_t y;
   asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(y) : "r"(x));
   return y;
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
