@@ -114,6 +114,19 @@ sd_status sd_attention_f16(const void* q, const void* k, const void* v, void* o,
                            void* stream);
 
 /*
+ * sd_attention with the element type and memory layout as arguments (an interface of this library:
+ * the layout a fused QKV projection writes, read without a transpose).
+ *  dtype  : 0 = bf16 (as sd_attention), 1 = fp16 (as sd_attention_f16).
+ *  layout : 0 = [B, heads, L, dh] (as sd_attention);
+ *           1 = [B, L, heads, dh] for q, k, v and o (heads interleaved in each row of the sequence;
+ *           read through a 4-D TMA tensor map, O written in the same layout).
+ * Other values of dtype or layout are SD_ERR_INVALID_ARG; everything else as in sd_attention.
+ */
+sd_status sd_attention_layout(const void* q, const void* k, const void* v, void* o,
+                              int64_t B, int64_t heads, int64_t Lq, int64_t Lk, int64_t dh, float scale,
+                              int dtype, int layout, void* stream);
+
+/*
  * sd_attention_noalloc -- the same computation, arguments, layouts and errors as sd_attention, for
  * callers that cannot allocate device memory. (The source pages have no counterpart: this is an
  * interface of this library.)

@@ -53,6 +53,14 @@ def test_attention_f16_argument_errors(L):
     assert L.sd_attention_f16(0, 0, 0, 0, 0, 1, 8, 8, 40, 1.0, None) == 0
 
 
+def test_attention_layout_argument_errors(L):
+    P = 1 << 12
+    assert L.sd_attention_layout(P, P + 4096, P + 8192, P + 12288, 1, 1, 8, 8, 40, 1.0, 2, 0, None) == 1  # dtype
+    assert L.sd_attention_layout(P, P + 4096, P + 8192, P + 12288, 1, 1, 8, 8, 40, 1.0, 0, 2, None) == 1  # layout
+    assert L.sd_attention_layout(P, P, P, P, 1, 1, 8, 8, 48, 1.0, 0, 1, None) == 2  # head dim
+    assert L.sd_attention_layout(0, 0, 0, 0, 0, 1, 8, 8, 40, 1.0, 1, 1, None) == 0
+
+
 def test_group_norm_argument_errors(L):
     P = 1 << 12
     assert L.sd_group_norm(P, P, P, P, 1, 30, 4, 4, 32, 1e-5, None) == 1  # 32 does not divide 30

@@ -175,3 +175,21 @@ def test_mixed_types_are_refused(cuda):
     q = torch.zeros(1, 1, 8, 40, dtype=torch.float16, device=cuda)
     with pytest.raises(ValueError):
         sdk.sd_attention(q, q.to(torch.bfloat16), q)
+
+
+# ---- [B, L, heads, dh] layout (sd_attention_layout, layout 1), bf16 and fp16
+
+@pytest.mark.parametrize("f16", [False, True], ids=["bf16", "fp16"])
+@pytest.mark.parametrize("dh,heads,Lq,Lk", [(40, 3, 300, 77), (64, 5, 513, 640), (80, 2, 129, 255), (160, 3, 200, 300),
+                                            (40, 80, 256, 640)])
+def test_blhd_layout(cuda, f16, dh, heads, Lq, Lk):
+    rnd = si.to_f16_exact if f16 else si.to_bf16_exact
+    seed = 13000 + dh + heads + Lk
+    q = rnd(si.normal((2, Lq, heads, dh), seed))
+    k = rnd(si.normal((2, Lk, heads, dh), seed + 1))
+    v = rnd(si.normal((2, Lk, heads, dh), seed + 2))
+    o = sdk.sd_attention(q.to(cuda), k.to(cuda), v.to(cuda), layout="blhd")
+    sdk.sd_device_status()
+    assert o.shape == q.shape and o.dtype == q.dtype
+    ref = oracle.attention(q.permute(0, 2, 1, 3), k.permute(0, 2, 1, 3), v.permute(0, 2, 1, 3))
+    _check(o.float().cpu().numpy().transpose(0, 2, 1, 3), ref)

@@ -53,12 +53,14 @@ def lib() -> ctypes.CDLL:
         L.sd_attention.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
         L.sd_attention_noalloc.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
         L.sd_attention_f16.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, vp]
+        L.sd_attention_layout.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, c_int, c_int, vp]
         L.sd_cfg_ddim_step.argtypes = [vp, vp, vp, vp, i64, f32, f64, f64, vp]
         L.sd_cfg_dpmpp_2m_step.argtypes = [vp, vp, vp, vp, vp, vp, i64, f32, f64, f64, f64, c_int, vp]
         L.sd_device_status.argtypes = [vp, c_int]
         L.sd_debug_set_fault.argtypes = [c_int]
         L.sd_debug_set_fault.restype = None
         for f in ("sd_group_norm", "sd_group_norm_silu", "sd_attention", "sd_attention_noalloc", "sd_attention_f16",
+                  "sd_attention_layout",
                   "sd_cfg_ddim_step",
                   "sd_cfg_dpmpp_2m_step", "sd_device_status"):
             getattr(L, f).restype = c_int
@@ -136,17 +138,27 @@ def sd_group_norm_silu(x, gamma, beta, groups: int = 32, eps: float = 1e-5, out=
     return out
 
 
-def sd_attention(q, k, v, scale: float | None = None, out=None):
-    """softmax(q k^T * scale) v for q [B,h,Lq,dh], k/v [B,h,Lk,dh], all bf16 or all fp16 (the output
-    has the same type); scale defaults to 1/sqrt(dh)."""
+def sd_attention(q, k, v, scale: float | None = None, out=None, layout: str = "bhld"):
+    """softmax(q k^T * scale) v for q [B,h,Lq,dh], k/v [B,h,Lk,dh] (layout "bhld") or q [B,Lq,h,dh],
+    k/v [B,Lk,h,dh] (layout "blhd"), all bf16 or all fp16 (the output has the type and layout of q);
+    scale defaults to 1/sqrt(dh)."""
     import torch
     if q.dtype not in (torch.bfloat16, torch.float16) or k.dtype != q.dtype or v.dtype != q.dtype:
         raise ValueError("sd_attention takes q, k, v all bf16 or all fp16")
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
-        raise ValueError("q, k, v must be [B, heads, L, dh]")
-    B, Hh, Lq, dh = q.shape
-    if k.shape[:2] != (B, Hh) or v.shape != k.shape or k.shape[3] != dh:
-        raise ValueError("k and v must be [B, heads, Lk, dh] matching q")
+        raise ValueError("q, k, v must be 4-D")
+    if layout not in ("bhld", "blhd"):
+        raise ValueError("layout must be 'bhld' or 'blhd'")
+    if layout == "blhd":
+        B, Lq, Hh, dh = q.shape
+        Lk = k.shape[1]
+        if k.shape != (B, Lk, Hh, dh) or v.shape != k.shape:
+            raise ValueError("k and v must be [B, Lk, heads, dh] matching q")
+    else:
+        B, Hh, Lq, dh = q.shape
+        Lk = k.shape[2]
+        if k.shape[:2] != (B, Hh) or v.shape != k.shape or k.shape[3] != dh:
+            raise ValueError("k and v must be [B, heads, Lk, dh] matching q")
     if out is None:
         out = torch.empty_like(q)
     _require_cuda(q, k, v, out)
@@ -154,9 +166,14 @@ def sd_attention(q, k, v, scale: float | None = None, out=None):
         raise ValueError("out must have the shape and type of q")
     if scale is None:
         scale = 1.0 / math.sqrt(dh)
-    name = "sd_attention_f16" if q.dtype == torch.float16 else "sd_attention"
-    _check(name, getattr(lib(), name)(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hh, Lq,
-                                      k.shape[2], dh, scale, _stream(q)))
+    f16, blhd = q.dtype == torch.float16, layout == "blhd"
+    if not f16 and not blhd:
+        st = lib().sd_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hh, Lq, Lk, dh, scale,
+                                _stream(q))
+    else:
+        st = lib().sd_attention_layout(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hh, Lq, Lk, dh,
+                                       scale, int(f16), int(blhd), _stream(q))
+    _check("sd_attention", st)
     return out
 
 

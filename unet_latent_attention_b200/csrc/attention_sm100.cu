@@ -260,6 +260,15 @@ __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile
 struct Seg {
   int it, kb, ke;
 };
+
+// One tile of rows [row, row + box) of head plane bh, 64 head-dim columns from x. lay_heads = 0:
+// tensors [B*heads, L, dh] (3-D map); lay_heads = heads: tensors [B, L, heads, dh] (4-D map over
+// {dh, heads, L, B}). Both put the same rows x 128 bytes into shared memory.
+__device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int row, int bh,
+                                          int lay_heads) {
+  if (lay_heads) tma_load_4d(dst, map, bar, x, bh % lay_heads, row, bh / lay_heads);
+  else tma_load_3d(dst, map, bar, x, row, bh);
+}
 __device__ __forceinline__ bool next_seg(long long& u, long long u1, int nkv, Seg& sg) {
   if (u >= u1) return false;
   sg.it = static_cast<int>(u / nkv);
@@ -275,7 +284,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out, int Lq, int Lk,
                    int dh, float scale_log2, unsigned int* err, int debug_flags, int qpairs, int items,
-                   float* __restrict__ ws, unsigned int* flags) {
+                   float* __restrict__ ws, unsigned int* flags, int lay_heads) {
   constexpr int BN = C::BN, NQ = C::NQ, STAGES = C::STAGES, NCH = C::NCH, NCHV = C::NCHV, DHP = C::DHP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -358,8 +367,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mbar_arrive_expect_tx(bars.q_full(qb), NQ * C::Q_TILE_BYTES);
         for (int t = 0; t < NQ; ++t)
           for (int c = 0; c < NCH; ++c)
-            tma_load_3d(sbase + C::Q_OFF + (qb * NQ + t) * C::Q_TILE_BYTES + c * BM * 128, &tm_q, bars.q_full(qb),
-                        c * 64, q0 + t * BM, bh);
+            load_rows(sbase + C::Q_OFF + (qb * NQ + t) * C::Q_TILE_BYTES + c * BM * 128, &tm_q, bars.q_full(qb),
+                      c * 64, q0 + t * BM, bh, lay_heads);
         ++nseg;
         for (int j = sg.kb; j < sg.ke; ++j, ++g) {
           const int s = g % STAGES, round = g / STAGES;
@@ -369,8 +378,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
           mbar_arrive_expect_tx(bars.k_full(s), C::K_TILE_BYTES);
           for (int c = 0; c < NCH; ++c)
-            tma_load_3d(sbase + C::K_OFF + s * C::K_TILE_BYTES + c * BN * 128, &tm_k, bars.k_full(s), c * 64,
-                        j * BN, bh);
+            load_rows(sbase + C::K_OFF + s * C::K_TILE_BYTES + c * BN * 128, &tm_k, bars.k_full(s), c * 64,
+                      j * BN, bh, lay_heads);
           issued[s] = round + 1;
           if ((debug_flags & 1) && g == 0) {  // test hook: the first V tile never arrives
             ok = false;
@@ -378,8 +387,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
           mbar_arrive_expect_tx(bars.v_full(s), C::V_TILE_BYTES);
           for (int c = 0; c < NCHV; ++c)
-            tma_load_3d(sbase + C::V_OFF + s * C::V_TILE_BYTES + c * BN * 128, &tm_v, bars.v_full(s), c * 64,
-                        j * BN, bh);
+            load_rows(sbase + C::V_OFF + s * C::V_TILE_BYTES + c * BN * 128, &tm_v, bars.v_full(s), c * 64,
+                      j * BN, bh, lay_heads);
         }
       }
       // Drain: every copy this thread issued has landed before the CTA may exit.
@@ -812,7 +821,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       packed[i] = C::F16 ? pack_f16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l)
                          : pack_bf16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l);
     if (qrow < Lq) {
-      uint4* dst = reinterpret_cast<uint4*>(out + (static_cast<size_t>(bh) * Lq + qrow) * dh);
+      const size_t orow = lay_heads ? (static_cast<size_t>(bh / lay_heads) * Lq + qrow) * lay_heads + bh % lay_heads
+                                    : static_cast<size_t>(bh) * Lq + qrow;
+      uint4* dst = reinterpret_cast<uint4*>(out + orow * dh);
       const int n16 = dh / 8;  // 16-byte groups of 8 bf16
 #pragma unroll
       for (int i = 0; i < DHP / 8; ++i)
@@ -844,16 +855,26 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 3-D map over a contiguous bf16 [planes, rows, dh] tensor, box {64, box_rows, 1}, 128-byte swizzle.
+// lay_heads = 0: [planes, rows, dh]; lay_heads = heads: [planes / heads, rows, heads, dh] as the 4-D
+// map {dh, heads, rows, B} with box {64, 1, box_rows, 1}.
 sd_status make_map(CUtensorMap* map, const void* ptr, int64_t dh, int64_t rows, int64_t planes, int box_rows,
-                   bool f16) {
+                   bool f16, int64_t lay_heads = 0) {
   auto fn = encode_fn();
   if (!fn) return sd::fail(SD_ERR_CUDA, "sd_attention: cuTensorMapEncodeTiled is unavailable");
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(dh), static_cast<cuuint64_t>(rows),
-                              static_cast<cuuint64_t>(planes)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(dh * 2), static_cast<cuuint64_t>(rows * dh * 2)};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+  const cuuint32_t rank = lay_heads ? 4 : 3;
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4];
+  if (lay_heads) {
+    dims[0] = dh, dims[1] = lay_heads, dims[2] = rows, dims[3] = planes / lay_heads;
+    strides[0] = dh * 2, strides[1] = lay_heads * dh * 2, strides[2] = rows * lay_heads * dh * 2;
+    box[0] = 64, box[1] = 1, box[2] = static_cast<cuuint32_t>(box_rows), box[3] = 1;
+  } else {
+    dims[0] = dh, dims[1] = rows, dims[2] = planes;
+    strides[0] = dh * 2, strides[1] = rows * dh * 2;
+    box[0] = 64, box[1] = static_cast<cuuint32_t>(box_rows), box[2] = 1;
+  }
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
                         const_cast<void*>(ptr), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -949,11 +970,11 @@ sd_status fixed_scratch(void** out) {
 // instead of the growable workspace, with its flags cleared on the stream first.
 template <class C>
 sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t BH, int64_t Lq, int64_t Lk,
-                 int64_t dh, float scale, cudaStream_t s, bool fixed = false) {
+                 int64_t dh, float scale, cudaStream_t s, bool fixed, int64_t lay_heads) {
   CUtensorMap mq, mk, mv;
-  sd_status st = make_map(&mq, q, dh, Lq, BH, BM, C::F16);
-  if (st == SD_OK) st = make_map(&mk, k, dh, Lk, BH, C::BN, C::F16);
-  if (st == SD_OK) st = make_map(&mv, v, dh, Lk, BH, C::BN, C::F16);
+  sd_status st = make_map(&mq, q, dh, Lq, BH, BM, C::F16, lay_heads);
+  if (st == SD_OK) st = make_map(&mk, k, dh, Lk, BH, C::BN, C::F16, lay_heads);
+  if (st == SD_OK) st = make_map(&mv, v, dh, Lk, BH, C::BN, C::F16, lay_heads);
   if (st != SD_OK) return st;
   unsigned int* err = sd::device_status_word();
   if (!err) return SD_ERR_CUDA;
@@ -1010,7 +1031,7 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
   return sd::cuda_check(
       cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, static_cast<uint16_t*>(o), static_cast<int>(Lq),
                          static_cast<int>(Lk), static_cast<int>(dh), scale_log2, err, g_debug_flags,
-                         static_cast<int>(qpairs), static_cast<int>(items), ws, flags),
+                         static_cast<int>(qpairs), static_cast<int>(items), ws, flags, static_cast<int>(lay_heads)),
       "sd_attention launch");
 }
 
@@ -1021,25 +1042,26 @@ namespace {
 // The launch table: a configuration per head dim and key length, for one element type.
 template <bool F16>
 sd_status dispatch(const void* q, const void* k, const void* v, void* o, int64_t BH, int64_t Lq, int64_t Lk,
-                   int64_t dh, float scale, cudaStream_t s, bool fixed) {
+                   int64_t dh, float scale, cudaStream_t s, bool fixed, int64_t lay_heads) {
   if (Lk <= 96) {  // short key sequence (the 77-token text context): one 96-key tile, no online rescale
     switch (dh) {
-      case 40: return launch<Cfg<40, 96, SD_CROSS_NQ, 2, true, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-      case 64: return launch<Cfg<64, 96, SD_CROSS_NQ, 2, true, false, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-      case 80: return launch<Cfg<80, 96, SD_CROSS_NQ, 2, true, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+      case 40: return launch<Cfg<40, 96, SD_CROSS_NQ, 2, true, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+      case 64: return launch<Cfg<64, 96, SD_CROSS_NQ, 2, true, false, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+      case 80: return launch<Cfg<80, 96, SD_CROSS_NQ, 2, true, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
       default: break;  // dh = 160 already uses 64-key tiles
     }
   }
   switch (dh) {
-    case 40: return launch<Cfg<40, 128, 2, SD_STAGES_SMALL, true, true, 2, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-    case 64: return launch<Cfg<64, 128, 2, SD_STAGES_SMALL, true, false, 2, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-    case 80: return launch<Cfg<80, 128, 2, 2, false, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
-    default: return launch<Cfg<160, 64, 1, 3, true, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+    case 40: return launch<Cfg<40, 128, 2, SD_STAGES_SMALL, true, true, 2, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+    case 64: return launch<Cfg<64, 128, 2, SD_STAGES_SMALL, true, false, 2, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+    case 80: return launch<Cfg<80, 128, 2, 2, false, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+    default: return launch<Cfg<160, 64, 1, 3, true, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
   }
 }
 
 sd_status attention_impl(const void* q, const void* k, const void* v, void* o, int64_t B, int64_t heads, int64_t Lq,
-                         int64_t Lk, int64_t dh, float scale, void* stream, bool fixed, bool f16 = false) {
+                         int64_t Lk, int64_t dh, float scale, void* stream, bool fixed, bool f16 = false,
+                         bool blhd = false) {
   if (B < 0 || heads < 0 || Lq < 0 || Lk < 0) return sd::fail(SD_ERR_INVALID_ARG, "sd_attention: negative size");
   if (dh != 40 && dh != 64 && dh != 80 && dh != 160)
     return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention: head dim %lld not in {40, 64, 80, 160}", (long long)dh);
@@ -1056,8 +1078,9 @@ sd_status attention_impl(const void* q, const void* k, const void* v, void* o, i
   if (sd::overlaps(o, qbytes, q, qbytes) || sd::overlaps(o, qbytes, k, kvbytes) || sd::overlaps(o, qbytes, v, kvbytes))
     return sd::fail(SD_ERR_INVALID_ARG, "sd_attention: o overlaps q, k or v");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return f16 ? dispatch<true>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed)
-             : dispatch<false>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed);
+  const int64_t lay_heads = blhd ? heads : 0;
+  return f16 ? dispatch<true>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads)
+             : dispatch<false>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
 }
 
 }  // namespace
@@ -1071,6 +1094,15 @@ extern "C" sd_status sd_attention(const void* q, const void* k, const void* v, v
 extern "C" sd_status sd_attention_f16(const void* q, const void* k, const void* v, void* o, int64_t B, int64_t heads,
                                       int64_t Lq, int64_t Lk, int64_t dh, float scale, void* stream) {
   return attention_impl(q, k, v, o, B, heads, Lq, Lk, dh, scale, stream, false, true);
+}
+
+// General entry: element type and memory layout as arguments (see sd_kernels.h).
+extern "C" sd_status sd_attention_layout(const void* q, const void* k, const void* v, void* o, int64_t B,
+                                         int64_t heads, int64_t Lq, int64_t Lk, int64_t dh, float scale, int dtype,
+                                         int layout, void* stream) {
+  if (dtype != 0 && dtype != 1) return sd::fail(SD_ERR_INVALID_ARG, "sd_attention_layout: dtype must be 0 or 1");
+  if (layout != 0 && layout != 1) return sd::fail(SD_ERR_INVALID_ARG, "sd_attention_layout: layout must be 0 or 1");
+  return attention_impl(q, k, v, o, B, heads, Lq, Lk, dh, scale, stream, false, dtype == 1, layout == 1);
 }
 
 // Same computation for callers that cannot allocate device memory (see sd_kernels.h): scratch comes
