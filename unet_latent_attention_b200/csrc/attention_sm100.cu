@@ -149,10 +149,14 @@ constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at B200 clocks
 // L_IN_V: the softmax row sums come out of the P V product itself: a fix-up warp writes bf16 1.0
 //         into column DH of every V tile once it lands (the TMA zero-fills columns >= DH), so O's
 //         column DH accumulates sum_j P_ij with no extra MMA (else fp32 adds in registers).
-// F16: the tensors (and P) are fp16 instead of bf16.
-template <int DH_, int BN_, int NQ_, int STAGES_, bool P_SEP_, bool L_IN_V_, int POLY_ = 0, bool F16_ = false>
+// F16: the tensors (and P) are fp16 instead of bf16. BLHD: the tensors are [B, L, heads, dh]
+// instead of [B, heads, L, dh] (a compile-time choice, so that the default layout's code is not
+// touched by the other's addressing).
+template <int DH_, int BN_, int NQ_, int STAGES_, bool P_SEP_, bool L_IN_V_, int POLY_ = 0, bool F16_ = false,
+          bool BLHD_ = false>
 struct Cfg {
   static constexpr bool F16 = F16_;
+  static constexpr bool BLHD = BLHD_;
   static constexpr int DH = DH_;          // true head dim
   static constexpr int DHP = (DH + 15) / 16 * 16;  // Q K^T depth padded to the MMA granule (16)
   static constexpr int BN = BN_;          // keys per K/V tile
@@ -264,9 +268,10 @@ struct Seg {
 // One tile of rows [row, row + box) of head plane bh, 64 head-dim columns from x. lay_heads = 0:
 // tensors [B*heads, L, dh] (3-D map); lay_heads = heads: tensors [B, L, heads, dh] (4-D map over
 // {dh, heads, L, B}). Both put the same rows x 128 bytes into shared memory.
+template <bool BLHD>
 __device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int row, int bh,
                                           int lay_heads) {
-  if (lay_heads) tma_load_4d(dst, map, bar, x, bh % lay_heads, row, bh / lay_heads);
+  if constexpr (BLHD) tma_load_4d(dst, map, bar, x, bh % lay_heads, row, bh / lay_heads);
   else tma_load_3d(dst, map, bar, x, row, bh);
 }
 __device__ __forceinline__ bool next_seg(long long& u, long long u1, int nkv, Seg& sg) {
@@ -367,7 +372,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mbar_arrive_expect_tx(bars.q_full(qb), NQ * C::Q_TILE_BYTES);
         for (int t = 0; t < NQ; ++t)
           for (int c = 0; c < NCH; ++c)
-            load_rows(sbase + C::Q_OFF + (qb * NQ + t) * C::Q_TILE_BYTES + c * BM * 128, &tm_q, bars.q_full(qb),
+            load_rows<C::BLHD>(sbase + C::Q_OFF + (qb * NQ + t) * C::Q_TILE_BYTES + c * BM * 128, &tm_q, bars.q_full(qb),
                       c * 64, q0 + t * BM, bh, lay_heads);
         ++nseg;
         for (int j = sg.kb; j < sg.ke; ++j, ++g) {
@@ -378,7 +383,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
           mbar_arrive_expect_tx(bars.k_full(s), C::K_TILE_BYTES);
           for (int c = 0; c < NCH; ++c)
-            load_rows(sbase + C::K_OFF + s * C::K_TILE_BYTES + c * BN * 128, &tm_k, bars.k_full(s), c * 64,
+            load_rows<C::BLHD>(sbase + C::K_OFF + s * C::K_TILE_BYTES + c * BN * 128, &tm_k, bars.k_full(s), c * 64,
                       j * BN, bh, lay_heads);
           issued[s] = round + 1;
           if ((debug_flags & 1) && g == 0) {  // test hook: the first V tile never arrives
@@ -387,7 +392,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
           mbar_arrive_expect_tx(bars.v_full(s), C::V_TILE_BYTES);
           for (int c = 0; c < NCHV; ++c)
-            load_rows(sbase + C::V_OFF + s * C::V_TILE_BYTES + c * BN * 128, &tm_v, bars.v_full(s), c * 64,
+            load_rows<C::BLHD>(sbase + C::V_OFF + s * C::V_TILE_BYTES + c * BN * 128, &tm_v, bars.v_full(s), c * 64,
                       j * BN, bh, lay_heads);
         }
       }
@@ -821,8 +826,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       packed[i] = C::F16 ? pack_f16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l)
                          : pack_bf16x2(ov[2 * i] * inv_l, ov[2 * i + 1] * inv_l);
     if (qrow < Lq) {
-      const size_t orow = lay_heads ? (static_cast<size_t>(bh / lay_heads) * Lq + qrow) * lay_heads + bh % lay_heads
-                                    : static_cast<size_t>(bh) * Lq + qrow;
+      const size_t orow = C::BLHD ? (static_cast<size_t>(bh / lay_heads) * Lq + qrow) * lay_heads + bh % lay_heads
+                                  : static_cast<size_t>(bh) * Lq + qrow;
       uint4* dst = reinterpret_cast<uint4*>(out + orow * dh);
       const int n16 = dh / 8;  // 16-byte groups of 8 bf16
 #pragma unroll
@@ -1040,22 +1045,22 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
 namespace {
 
 // The launch table: a configuration per head dim and key length, for one element type.
-template <bool F16>
+template <bool F16, bool BLHD>
 sd_status dispatch(const void* q, const void* k, const void* v, void* o, int64_t BH, int64_t Lq, int64_t Lk,
                    int64_t dh, float scale, cudaStream_t s, bool fixed, int64_t lay_heads) {
   if (Lk <= 96) {  // short key sequence (the 77-token text context): one 96-key tile, no online rescale
     switch (dh) {
-      case 40: return launch<Cfg<40, 96, SD_CROSS_NQ, 2, true, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
-      case 64: return launch<Cfg<64, 96, SD_CROSS_NQ, 2, true, false, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
-      case 80: return launch<Cfg<80, 96, SD_CROSS_NQ, 2, true, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+      case 40: return launch<Cfg<40, 96, SD_CROSS_NQ, 2, true, true, 0, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+      case 64: return launch<Cfg<64, 96, SD_CROSS_NQ, 2, true, false, 0, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+      case 80: return launch<Cfg<80, 96, SD_CROSS_NQ, 2, true, true, 0, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
       default: break;  // dh = 160 already uses 64-key tiles
     }
   }
   switch (dh) {
-    case 40: return launch<Cfg<40, 128, 2, SD_STAGES_SMALL, true, true, 2, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
-    case 64: return launch<Cfg<64, 128, 2, SD_STAGES_SMALL, true, false, 2, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
-    case 80: return launch<Cfg<80, 128, 2, 2, false, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
-    default: return launch<Cfg<160, 64, 1, 3, true, true, 0, F16>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+    case 40: return launch<Cfg<40, 128, 2, SD_STAGES_SMALL, true, true, 2, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+    case 64: return launch<Cfg<64, 128, 2, SD_STAGES_SMALL, true, false, 2, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+    case 80: return launch<Cfg<80, 128, 2, 2, false, true, 0, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+    default: return launch<Cfg<160, 64, 1, 3, true, true, 0, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
   }
 }
 
@@ -1079,8 +1084,11 @@ sd_status attention_impl(const void* q, const void* k, const void* v, void* o, i
     return sd::fail(SD_ERR_INVALID_ARG, "sd_attention: o overlaps q, k or v");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int64_t lay_heads = blhd ? heads : 0;
-  return f16 ? dispatch<true>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads)
-             : dispatch<false>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+  if (blhd)
+    return f16 ? dispatch<true, true>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads)
+               : dispatch<false, true>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+  return f16 ? dispatch<true, false>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads)
+             : dispatch<false, false>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
 }
 
 }  // namespace
