@@ -106,6 +106,10 @@ constexpr int kTraceLast = 0;
 #define SD_EXP_BF16 0  // tuning: exp2 of bf16 pairs on the special-function unit (see the exp loop)
 #endif
 
+#ifndef SD_L2_PREFETCH
+#define SD_L2_PREFETCH 0  // prefetch the first tiles into L2 before waiting for the previous kernel
+#endif
+
 #ifndef SD_P_CHUNKED
 #define SD_P_CHUNKED -1  // tuning override of Cfg::CHUNK_P (-1: the per-config choice)
 #endif
@@ -269,6 +273,12 @@ struct Seg {
 // tensors [B*heads, L, dh] (3-D map); lay_heads = heads: tensors [B, L, heads, dh] (4-D map over
 // {dh, heads, L, B}). Both put the same rows x 128 bytes into shared memory.
 template <bool BLHD>
+__device__ __forceinline__ void prefetch_rows(const CUtensorMap* map, int x, int row, int bh, int lay_heads) {
+  if constexpr (BLHD) tma_prefetch_4d(map, x, bh % lay_heads, row, bh / lay_heads);
+  else tma_prefetch_3d(map, x, row, bh);
+}
+
+template <bool BLHD>
 __device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int row, int bh,
                                           int lay_heads) {
   if constexpr (BLHD) tma_load_4d(dst, map, bar, x, bh % lay_heads, row, bh / lay_heads);
@@ -344,7 +354,20 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // Everything above touched only shared memory, tensor memory and the kernel parameters: it may
-  // overlap the end of the previous kernel on the stream. Global memory waits for that kernel.
+  // overlap the end of the previous kernel on the stream. Global memory waits for that kernel; an
+  // L2 prefetch of this CTA's first Q tiles and K/V tiles is only a hint (it returns no data, and
+  // the loads after the wait read whatever the previous kernel wrote), so it goes first.
+  if (SD_L2_PREFETCH && threadIdx.x == 0 && u0 < u1) {
+    const int it = static_cast<int>(u0 / nkv), kb = static_cast<int>(u0 % nkv);
+    const int bh = it / qpairs, q0 = (it % qpairs) * (BM * NQ);
+    for (int t = 0; t < NQ; ++t)
+      for (int c = 0; c < NCH; ++c) prefetch_rows<C::BLHD>(&tm_q, c * 64, q0 + t * BM, bh, lay_heads);
+    const int ke = static_cast<int>(kb + STAGES < nkv ? kb + STAGES : nkv);
+    for (int j = kb; j < ke && j < kb + (u1 - u0); ++j) {
+      for (int c = 0; c < NCH; ++c) prefetch_rows<C::BLHD>(&tm_k, c * 64, j * BN, bh, lay_heads);
+      for (int c = 0; c < NCHV; ++c) prefetch_rows<C::BLHD>(&tm_v, c * 64, j * BN, bh, lay_heads);
+    }
+  }
   sd::grid_dep_wait();
   sd::grid_dep_launch();
   if (threadIdx.x == 0) SD_SEG(0);
