@@ -34,7 +34,10 @@
 #include <atomic>
 #include <algorithm>
 #include <cmath>
+#include <map>
 #include <mutex>
+#include <tuple>
+#include <vector>
 
 #include "sd_internal.h"
 #include "sm100_ptx.cuh"
@@ -212,6 +215,9 @@ struct Cfg {
   // Store P in 16-column chunks inside the exp2 loop (measured: faster for the single short key
   // tile of cross-attention, slower for the long key loops).
   static constexpr bool CHUNK_P = BN < 128;
+  // Costs of the persistent schedule in K/V-tile units (measured; see part_ranges).
+  static constexpr double COST_SEG = DH == 64 ? 1.3 : 1.0, COST_TAIL = DH == 64 ? 0.5 : 0.6,
+                          COST_HEAD = DH == 64 ? 1.4 : 0.9;
   // Of every 8 column pairs, this many take the FMA-pipe exp2 instead of the special-function unit.
   static constexpr int POLY_PAIRS = SD_POLY_PAIRS >= 0 ? SD_POLY_PAIRS : POLY_;
   static_assert(NPV % 16 == 0 && NPV <= 256, "MMA N must be a multiple of 16 and at most 256");
@@ -269,6 +275,13 @@ struct Seg {
   int it, kb, ke;
 };
 
+// Unit ranges of the persistent grid: CTA c owns units [u[c], u[c+1]). Passed by value (kernel
+// parameter space), filled on the host: evenly, or balanced by a cost model (see part_ranges).
+constexpr int kMaxCtas = 256;
+struct Part {
+  long long u[kMaxCtas + 1];
+};
+
 // One tile of rows [row, row + box) of head plane bh, 64 head-dim columns from x. lay_heads = 0:
 // tensors [B*heads, L, dh] (3-D map); lay_heads = heads: tensors [B, L, heads, dh] (4-D map over
 // {dh, heads, L, B}). Both put the same rows x 128 bytes into shared memory.
@@ -299,7 +312,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out, int Lq, int Lk,
                    int dh, float scale_log2, unsigned int* err, int debug_flags, int qpairs, int items,
-                   float* __restrict__ ws, unsigned int* flags, int lay_heads) {
+                   float* __restrict__ ws, unsigned int* flags, int lay_heads,
+                   const __grid_constant__ Part part) {
   constexpr int BN = C::BN, NQ = C::NQ, STAGES = C::STAGES, NCH = C::NCH, NCHV = C::NCHV, DHP = C::DHP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -310,8 +324,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkv = (Lk + BN - 1) / BN;
-  const long long U = static_cast<long long>(items) * nkv;
-  const long long u0 = U * blockIdx.x / gridDim.x, u1 = U * (blockIdx.x + 1) / gridDim.x;
+  const long long u0 = part.u[blockIdx.x], u1 = part.u[blockIdx.x + 1];
 
   if (threadIdx.x == 0) SD_TR(0, kTraceLast, 0);  // kernel entry (tuning builds only)
   SD_SPAN_DECL;
@@ -994,6 +1007,81 @@ sd_status fixed_scratch(void** out) {
   return SD_OK;
 }
 
+#ifndef SD_BALANCE
+#define SD_BALANCE 1  // unit ranges balanced by the cost model below (0: equal unit counts)
+#endif
+
+// Per-CTA unit ranges. Equal unit counts leave CTAs with more segment boundaries, or ending in a
+// split item's merge, finishing last. Measured on B200 with global-timer spans (SD1.5 and SDXL
+// shapes), in K/V-tile units: each segment boundary costs about 1.0 tile, publishing a tail piece
+// 0.6, merging a head piece 0.9 (dh 40; 1.3, 0.5 and 1.4 for dh 64). The range of each CTA is
+// chosen so that tiles plus these costs stay below the smallest bound T that covers all units;
+// a range never lies strictly inside one item, so an item still spans at most two consecutive
+// CTAs. Results are cached per shape.
+struct CostModel {
+  double seg, tail, head;
+};
+
+double range_cost(long long a, long long b, long long nkv, const CostModel& m) {
+  const long long segs = (b - 1) / nkv - a / nkv + 1;
+  return static_cast<double>(b - a) + m.seg * static_cast<double>(segs - 1) + (a % nkv ? m.tail : 0.0) +
+         (b % nkv ? m.head : 0.0);
+}
+
+bool inside_one_item(long long a, long long b, long long nkv) {
+  return a % nkv != 0 && b % nkv != 0 && a / nkv == (b - 1) / nkv;
+}
+
+bool fill_ranges(long long U, long long nkv, int G, const CostModel& m, double T, long long* u) {
+  long long a = 0;
+  u[0] = 0;
+  for (int c = 0; c < G; ++c) {
+    if (a >= U) {
+      u[c + 1] = U;
+      continue;
+    }
+    long long best = -1;
+    const long long hi = std::min<long long>(U, a + static_cast<long long>(T) + 1);
+    for (long long b = hi; b > a && b + 64 > hi; --b)
+      if (!inside_one_item(a, b, nkv) && range_cost(a, b, nkv, m) <= T) {
+        best = b;
+        break;
+      }
+    if (best < 0) return false;
+    u[c + 1] = best;
+    a = best;
+  }
+  return a == U;
+}
+
+void part_ranges(long long U, long long nkv, int G, const CostModel& m, long long* u) {
+  auto even = [&] {
+    for (int c = 0; c <= G; ++c) u[c] = U * c / G;
+  };
+  if (!SD_BALANCE || nkv <= 1) return even();
+  static std::mutex mu;
+  static std::map<std::tuple<long long, long long, int, double, double, double>, std::vector<long long>> cache;
+  const auto key = std::make_tuple(U, nkv, G, m.seg, m.tail, m.head);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it == cache.end()) {
+    std::vector<long long> v(G + 1);
+    double lo = static_cast<double>(U) / G, hi = lo + 4.0 * (m.seg + m.tail + m.head) + 2.0;
+    if (!fill_ranges(U, nkv, G, m, hi, v.data())) {
+      for (int c = 0; c <= G; ++c) v[c] = U * c / G;  // no balanced split found: equal counts
+    } else {
+      for (int i = 0; i < 40; ++i) {  // smallest T (to 1e-3 tiles) that still covers all units
+        const double mid = 0.5 * (lo + hi);
+        if (fill_ranges(U, nkv, G, m, mid, v.data())) hi = mid;
+        else lo = mid;
+      }
+      fill_ranges(U, nkv, G, m, hi, v.data());
+    }
+    it = cache.emplace(key, std::move(v)).first;
+  }
+  std::copy(it->second.begin(), it->second.end(), u);
+}
+
 // `fixed` selects the caller-side contract of sd_attention_noalloc: scratch from g_fixed_scratch
 // instead of the growable workspace, with its flags cleared on the stream first.
 template <class C>
@@ -1023,7 +1111,7 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
   const int64_t qpairs = (Lq + BM * C::NQ - 1) / (BM * C::NQ);
   const int64_t items = BH * qpairs;
   const int64_t nkv = (Lk + C::BN - 1) / C::BN;
-  const int64_t G = std::min<int64_t>(sd::sm_count(), items);
+  const int64_t G = std::min<int64_t>(std::min<int64_t>(sd::sm_count(), items), kMaxCtas);
   if (items > 0x7fffffff || items * nkv > (int64_t(1) << 40))
     return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention: too many tiles");
   float* ws = nullptr;
@@ -1047,6 +1135,8 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
     ws = static_cast<float*>(p);
     flags = reinterpret_cast<unsigned int*>(static_cast<char*>(p) + fbytes);
   }
+  Part part;
+  part_ranges(items * nkv, nkv, static_cast<int>(G), CostModel{C::COST_SEG, C::COST_TAIL, C::COST_HEAD}, part.u);
   const float scale_log2 = scale * 1.4426950408889634f;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(G));
@@ -1059,7 +1149,8 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
   return sd::cuda_check(
       cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, static_cast<uint16_t*>(o), static_cast<int>(Lq),
                          static_cast<int>(Lk), static_cast<int>(dh), scale_log2, err, g_debug_flags,
-                         static_cast<int>(qpairs), static_cast<int>(items), ws, flags, static_cast<int>(lay_heads)),
+                         static_cast<int>(qpairs), static_cast<int>(items), ws, flags, static_cast<int>(lay_heads),
+                         part),
       "sd_attention launch");
 }
 
