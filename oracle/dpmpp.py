@@ -15,7 +15,9 @@ parametrisation on the cumulative products alpha_bar:
     order 2:  r = (lambda_t - lambda_prev) / h,
               x' = (sigma_next / sigma_t) x - alpha_next (exp(-h) - 1) ((1 + 1/(2r)) D - 1/(2r) D_prev)
 
-where D_prev is the data prediction of the previous step (the history). The step to
+where D_prev is the data prediction of the previous step (the history). Order 3 (the page's
+"三阶") is the third-order multistep update of the same family on two history entries
+(dpmpp_3m_step). The step to
 alpha_bar = 1 (sigma = 0, the end of sampling) is taken at first order and returns D. Karras
 sigmas (Karras et al. 2022, rho = 7) span the Stable Diffusion scaled-linear range and map to
 alpha_bar = 1 / (1 + sigma^2).
@@ -60,10 +62,46 @@ def dpmpp_2m_step(x, g, d_prev, alpha_prev: float, alpha_t: float, alpha_next: f
     return (s_n / s_t) * x - a_n * np.expm1(-h) * Dhat, D
 
 
+def dpmpp_3m_step(x, g, d1, d2, alpha_p2: float, alpha_p1: float, alpha_t: float, alpha_next: float):
+    """Third-order multistep DPM-Solver++ step; returns (x_next, D).
+
+    d1, d2 are the data predictions of the previous two steps, taken at alpha_bar = alpha_p1 and
+    alpha_p2. With m0 = D, m1 = d1, m2 = d2, h = lambda_next - lambda_t, h0 = lambda_t - lambda_p1,
+    h1 = lambda_p1 - lambda_p2, r0 = h0 / h, r1 = h1 / h:
+        D1_0 = (m0 - m1) / r0,  D1_1 = (m1 - m2) / r1
+        D1   = D1_0 + r0 / (r0 + r1) (D1_0 - D1_1)      h * D'(lambda_t) of the quadratic through m2, m1, m0
+        D2   = (D1_0 - D1_1) / (r0 + r1)                h^2 * D''/2 of that quadratic
+        x'   = (sigma_next / sigma_t) x - alpha_next (e^-h - 1) m0
+               + alpha_next ((e^-h - 1) / h + 1) D1 - 2 alpha_next ((e^-h - 1 + h) / h^2 - 1/2) D2
+    This is the exact integral x' = (sigma_next/sigma_t) x + sigma_next int e^lambda D(lambda) dlambda
+    of the quadratic that interpolates the three data predictions in lambda (the multistep
+    third-order construction of DPM-Solver, Lu et al. 2022, in data-prediction form), hence
+    third-order accurate."""
+    x = np.asarray(x, np.float64)
+    m0 = data_prediction(x, g, alpha_t)
+    m1, m2 = np.asarray(d1, np.float64), np.asarray(d2, np.float64)
+    a_n, s_n, s_t = np.sqrt(alpha_next), np.sqrt(1.0 - alpha_next), np.sqrt(1.0 - alpha_t)
+    h = lam(alpha_next) - lam(alpha_t)
+    r0 = (lam(alpha_t) - lam(alpha_p1)) / h
+    r1 = (lam(alpha_p1) - lam(alpha_p2)) / h
+    d1_0, d1_1 = (m0 - m1) / r0, (m1 - m2) / r1
+    D1 = d1_0 + r0 / (r0 + r1) * (d1_0 - d1_1)
+    D2 = (d1_0 - d1_1) / (r0 + r1)
+    em = np.expm1(-h)
+    xn = ((s_n / s_t) * x - a_n * em * m0 + a_n * (em / h + 1.0) * D1 - 2.0 * a_n * ((em + h) / h ** 2 - 0.5) * D2)
+    return xn, m0
+
+
 def cfg_dpmpp_2m_step(x, eps_u, eps_c, d_prev, w: float, alpha_prev: float, alpha_t: float, alpha_next: float,
                       order: int):
     """One guided step: DPM-Solver++ on the CFG-combined noise prediction; returns (x_next, D)."""
     return dpmpp_2m_step(x, cfg(eps_u, eps_c, w), d_prev, alpha_prev, alpha_t, alpha_next, order)
+
+
+def cfg_dpmpp_3m_step(x, eps_u, eps_c, d1, d2, w: float, alpha_p2: float, alpha_p1: float, alpha_t: float,
+                      alpha_next: float):
+    """Guided third-order multistep step; returns (x_next, D)."""
+    return dpmpp_3m_step(x, cfg(eps_u, eps_c, w), d1, d2, alpha_p2, alpha_p1, alpha_t, alpha_next)
 
 
 def karras_sigmas(n: int, sigma_min: float, sigma_max: float, rho: float = 7.0) -> np.ndarray:

@@ -109,3 +109,60 @@ def test_schedule_and_loop_end_on_the_data():
         g = (x - np.sqrt(a_t) * x0) / np.sqrt(1 - a_t)
         x, d = oracle.dpmpp_2m_step(x, g, d, a_p, a_t, a_n, order)
     np.testing.assert_allclose(x, x0, rtol=1e-10, atol=1e-10)
+
+
+# ---- third order (two history entries)
+
+def _solve3(n, D, x_start=2.0, l0=-1.5, l1=1.5):
+    """n third-order steps, uniform in lambda, on the data prediction D(lambda). The history starts
+    from the model's values at two points before l0 (a lower-order warm-up would cap the global
+    order at its own)."""
+    h = (l1 - l0) / n
+    lams = l0 + h * np.arange(-2, n + 1)  # lams[2] = l0
+    x, hist = np.array([x_start]), [D(lams[0]), D(lams[1])]
+    for i in range(2, n + 2):
+        a_t, a_n = _alpha_bar_of_lambda(lams[i]), _alpha_bar_of_lambda(lams[i + 1])
+        g = (x - np.sqrt(a_t) * D(lams[i])) / np.sqrt(1 - a_t)
+        x, d = oracle.dpmpp_3m_step(x, g, hist[-1], hist[-2], _alpha_bar_of_lambda(lams[i - 2]),
+                                    _alpha_bar_of_lambda(lams[i - 1]), a_t, a_n)
+        hist.append(d)
+    return x[0]
+
+
+def _exact_F(F, x_start=2.0, l0=-1.5, l1=1.5):
+    """x(l1) for the data prediction whose integral against e^u is F: (sigma1/sigma0) x0 + sigma1 (F(l1) - F(l0))."""
+    sig = lambda l: np.sqrt(1 - _alpha_bar_of_lambda(l))
+    return sig(l1) / sig(l0) * x_start + sig(l1) * (F(l1) - F(l0))
+
+
+def test_third_order_is_exact_on_a_quadratic_data_prediction():
+    # the step integrates e^lambda times the quadratic through three data predictions exactly
+    c = (0.7, -1.3, 0.9)
+    D = lambda l: c[0] + c[1] * l + c[2] * l * l
+    F = lambda u: np.exp(u) * (c[0] + c[1] * (u - 1) + c[2] * (u * u - 2 * u + 2))  # int e^u D(u) du
+    for n in (5, 17):
+        assert abs(_solve3(n, D) - _exact_F(F)) < 1e-12
+
+
+def test_third_order_convergence():
+    D = lambda l: np.sin(2 * l)
+    F = lambda u: np.exp(u) * (np.sin(2 * u) - 2 * np.cos(2 * u)) / 5  # int e^u sin(2u) du
+    e3 = [abs(_solve3(n, D) - _exact_F(F)) for n in (80, 160, 320)]  # asymptotic regime
+    for a, b in zip(e3, e3[1:]):
+        assert 6.5 < a / b < 9.5, e3
+
+
+def test_third_order_reproduces_a_linear_data_prediction_exactly_up_to_the_warm_up():
+    # third-order divided differences of a linear D vanish; from the same starting point the
+    # third-order step and the exact exponential integral then differ only through D1's model
+    # a_p2, a_p1, a_t, a_n spaced evenly in lambda; D linear => D2 = 0 and D1 = slope * h exactly
+    ls = np.array([-1.0, -0.7, -0.4, -0.1])
+    ab = [_alpha_bar_of_lambda(l) for l in ls]
+    Dl = lambda l: 0.3 + 0.8 * l
+    x = np.array([1.25])
+    g = (x - np.sqrt(ab[2]) * Dl(ls[2])) / np.sqrt(1 - ab[2])
+    xn, _ = oracle.dpmpp_3m_step(x, g, Dl(ls[1]), Dl(ls[0]), ab[0], ab[1], ab[2], ab[3])
+    sig = lambda l: np.sqrt(1 - _alpha_bar_of_lambda(l))
+    F = lambda u: np.exp(u) * (0.3 + 0.8 * (u - 1))
+    exact = sig(ls[3]) / sig(ls[2]) * x + sig(ls[3]) * (F(ls[3]) - F(ls[2]))
+    np.testing.assert_allclose(xn, exact, rtol=1e-12)
