@@ -377,6 +377,21 @@ def bench_extra(sdk, dev, hbm):
     byts = sum(24 if o == 2 else 20 for *_, o in dsched) * n
     out["cfg_dpmpp_2m_20_steps_serving"] = {"shape": list(lat), "us_per_loop": us, "us_per_step": us / 20,
                                             "GB/s": byts / (us * 1e-6) / 1e9}
+    # third-order multistep run (orders 1, 2, 3, ..., 3, 1), history rotated through three buffers
+    bufs = [torch.zeros(lat, device=dev) for _ in range(3)]
+    tsched = sdk.dpmpp_3m_schedule(20)
+
+    def loop3(_):
+        for i, ((a2, a1, a_t, a_n, order), (eu, ec)) in enumerate(zip(tsched, eps)):
+            d_out, d1, d2 = bufs[i % 3], bufs[(i - 1) % 3], bufs[(i - 2) % 3]
+            if order == 3:
+                sdk.sd_cfg_dpmpp_3m_step(x, eu, ec, d1, d2, 7.5, a2, a1, a_t, a_n, out=x, d_out=d_out)
+            else:
+                sdk.sd_cfg_dpmpp_2m_step(x, eu, ec, d1, 7.5, a1, a_t, a_n, order, out=x, d_out=d_out)
+    us = _graph_time_us(loop3, 5, dev)
+    byts = sum({1: 20, 2: 24, 3: 28}[o] for *_, o in tsched) * n
+    out["cfg_dpmpp_3m_20_steps_serving"] = {"shape": list(lat), "us_per_loop": us, "us_per_step": us / 20,
+                                            "GB/s": byts / (us * 1e-6) / 1e9}
     sweep = []
     for (B, C, H, W) in [(2, 320, 64, 64), (8, 320, 96, 96), (16, 640, 64, 64), (16, 320, 128, 128)]:
         xs = [torch.randn(B, C, H, W, device=dev) for _ in range(2)]

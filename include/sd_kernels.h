@@ -194,6 +194,28 @@ sd_status sd_cfg_dpmpp_2m_step(const float* x, const float* eps_u, const float* 
                                float* x_out, float* d_out, int64_t n, float w, double alpha_prev,
                                double alpha_t, double alpha_next, int order, void* stream);
 
+/*
+ * Guided third-order multistep DPM-Solver++ step (the engine page's order 3, §4). With
+ * m0 = D = (x - sigma_t g) / alpha_t, m1 = d_prev (taken at alpha_prev), m2 = d_prev2 (at
+ * alpha_prev2), h = lambda_next - lambda_t, r0 = (lambda_t - lambda_prev) / h,
+ * r1 = (lambda_prev - lambda_prev2) / h:
+ *   D1_0 = (m0 - m1) / r0, D1_1 = (m1 - m2) / r1,
+ *   D1 = D1_0 + r0 / (r0 + r1) (D1_0 - D1_1), D2 = (D1_0 - D1_1) / (r0 + r1),
+ *   x' = (sigma_next / sigma_t) x - alpha_next expm1(-h) m0 + alpha_next (expm1(-h) / h + 1) D1
+ *        - 2 alpha_next ((expm1(-h) + h) / h^2 - 1/2) D2,
+ * the exact exponential integral of the quadratic through (lambda, m) of the three steps.
+ *  x, eps_u, eps_c, x_out : as in sd_cfg_dpmpp_2m_step.
+ *  d_prev, d_prev2 : fp32 n, the data predictions of the previous two steps.
+ *  d_out  : fp32 n, this step's D; may equal d_prev or d_prev2 (the caller rotates the history).
+ *  alpha_prev2, alpha_prev, alpha_t, alpha_next : in (0, 1), pairwise distinct in lambda; the step
+ *           to alpha_bar = 1 is first order (sd_cfg_dpmpp_2m_step with order 1).
+ * Other values, NULL pointers and other overlaps are SD_ERR_INVALID_ARG.
+ */
+sd_status sd_cfg_dpmpp_3m_step(const float* x, const float* eps_u, const float* eps_c, const float* d_prev,
+                               const float* d_prev2, float* x_out, float* d_out, int64_t n, float w,
+                               double alpha_prev2, double alpha_prev, double alpha_t, double alpha_next,
+                               void* stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* sd_status_string(sd_status status);
 

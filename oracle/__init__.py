@@ -30,9 +30,10 @@ from .ddim import (cfg, ddim_step, cfg_ddim_step, scaled_linear_betas, alphas_cu
                    ddim_timesteps, ddim_schedule, cfg_ddim_loop)
 from .dpmpp import (lam, data_prediction, dpmpp_2m_step, cfg_dpmpp_2m_step, dpmpp_3m_step, cfg_dpmpp_3m_step,
                     karras_sigmas, alpha_bar_of_sigma,
-                    sd_sigma_range, dpmpp_2m_schedule, cfg_dpmpp_2m_loop)
+                    sd_sigma_range, dpmpp_2m_schedule, cfg_dpmpp_2m_loop, dpmpp_3m_schedule, cfg_dpmpp_3m_loop)
 
 __all__ = ["attention", "attention_rows", "softmax_weights", "group_norm", "group_norm_silu", "group_stats",
            "silu", "cfg", "ddim_step", "cfg_ddim_step", "scaled_linear_betas", "alphas_cumprod", "ddim_timesteps",
            "ddim_schedule", "cfg_ddim_loop", "lam", "data_prediction", "dpmpp_2m_step", "cfg_dpmpp_2m_step",
-           "dpmpp_3m_step", "cfg_dpmpp_3m_step", "karras_sigmas", "alpha_bar_of_sigma", "sd_sigma_range", "dpmpp_2m_schedule", "cfg_dpmpp_2m_loop"]
+           "dpmpp_3m_step", "cfg_dpmpp_3m_step", "karras_sigmas", "alpha_bar_of_sigma", "sd_sigma_range", "dpmpp_2m_schedule", "cfg_dpmpp_2m_loop",
+           "dpmpp_3m_schedule", "cfg_dpmpp_3m_loop"]

@@ -143,3 +143,27 @@ def cfg_dpmpp_2m_loop(x, eps_pairs, w: float, schedule):
     for (a_p, a_t, a_n, order), (eu, ec) in zip(schedule, eps_pairs):
         x, d = cfg_dpmpp_2m_step(x, eu, ec, d, w, a_p, a_t, a_n, order)
     return x
+
+
+def dpmpp_3m_schedule(steps: int = 20):
+    """[(alpha_prev2, alpha_prev, alpha_t, alpha_next, order)]: orders 1, 2, then 3; last step order 1."""
+    smin, smax = sd_sigma_range()
+    ab = list(alpha_bar_of_sigma(karras_sigmas(steps, smin, smax))) + [1.0]
+    out = []
+    for i in range(steps):
+        order = 1 if i == 0 or i == steps - 1 else min(i + 1, 3)
+        out.append((ab[i - 2] if i >= 2 else ab[i], ab[i - 1] if i >= 1 else ab[i], ab[i], ab[i + 1], order))
+    return out
+
+
+def cfg_dpmpp_3m_loop(x, eps_pairs, w: float, schedule):
+    """Runs a guided multistep run of orders 1-3 (schedule from dpmpp_3m_schedule)."""
+    x = np.asarray(x, np.float64)
+    hist = []
+    for (a_p2, a_p1, a_t, a_n, order), (eu, ec) in zip(schedule, eps_pairs):
+        if order == 3:
+            x, d = cfg_dpmpp_3m_step(x, eu, ec, hist[-1], hist[-2], w, a_p2, a_p1, a_t, a_n)
+        else:
+            x, d = cfg_dpmpp_2m_step(x, eu, ec, hist[-1] if hist else None, w, a_p1, a_t, a_n, order)
+        hist.append(d)
+    return x

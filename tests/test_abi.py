@@ -101,12 +101,27 @@ def test_dpmpp_argument_errors(L):
     assert f(0, 0, 0, 0, 0, 0, 0, 7.5, 0.2, 0.3, 0.4, 1, None) == 0  # empty
 
 
+def test_dpmpp_3m_argument_errors(L):
+    P, n = 1 << 12, 16
+    Q = [P + i * 4096 for i in range(7)]  # x, eu, ec, d_prev, d_prev2, x_out, d_out: disjoint
+    f = L.sd_cfg_dpmpp_3m_step
+    assert f(*Q, n, 7.5, 0.1, 0.2, 0.3, 1.0, None) == 1 and "first order" in _err(L)  # to sigma = 0
+    assert f(*Q, n, 7.5, 0.2, 0.2, 0.3, 0.4, None) == 1  # equal noise levels
+    assert f(Q[0], Q[1], Q[2], 0, Q[4], Q[5], Q[6], n, 7.5, 0.1, 0.2, 0.3, 0.4, None) == 1  # null history
+    assert f(Q[0], Q[1], Q[2], Q[3], Q[4], Q[5], Q[3] + 4, n, 7.5, 0.1, 0.2, 0.3, 0.4, None) == 1  # partial alias
+    assert f(Q[0], Q[1], Q[2], Q[3], Q[4], Q[5], Q[4], 0, 7.5, 0.1, 0.2, 0.3, 0.4, None) == 0  # d_out == d_prev2
+
+
 def test_dpmpp_schedule_matches_the_oracle():
     import oracle
     ours, ref = sdk.dpmpp_2m_schedule(20), oracle.dpmpp_2m_schedule(20)
     assert [o for *_, o in ours] == [o for *_, o in ref]
     for a, b in zip(ours, ref):
         assert max(abs(x - y) for x, y in zip(a[:3], b[:3])) < 1e-13
+    ours, ref = sdk.dpmpp_3m_schedule(20), oracle.dpmpp_3m_schedule(20)
+    assert [o for *_, o in ours] == [o for *_, o in ref]
+    for a, b in zip(ours, ref):
+        assert max(abs(x - y) for x, y in zip(a[:4], b[:4])) < 1e-13
 
 
 def test_binding_refuses_cpu_tensors(L):

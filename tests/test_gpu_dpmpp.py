@@ -74,3 +74,38 @@ def test_twenty_step_sampling_run(cuda):
     sdk.sd_device_status()
     ref = oracle.cfg_dpmpp_2m_loop(x0, eps, W, oracle.dpmpp_2m_schedule(20))
     assert rel_err(xd.cpu().numpy(), ref) <= REL_LOOP
+
+
+# ---- third order
+
+@pytest.mark.parametrize("alphas", [(0.01, 0.02, 0.035, 0.05), (0.3, 0.35, 0.4, 0.45), (0.8, 0.88, 0.93, 0.97)])
+@pytest.mark.parametrize("shape", [(8, 4, 96, 96), (3, 5, 7, 11)])
+def test_third_order_step(cuda, alphas, shape):
+    x, eu, ec, d1 = _inputs(shape, 1600 + sum(shape))
+    d2 = si.normal(shape, 1700 + sum(shape))
+    a2, a1, a_t, a_n = alphas
+    xo, d = sdk.sd_cfg_dpmpp_3m_step(_t(x, cuda), _t(eu, cuda), _t(ec, cuda), _t(d1, cuda), _t(d2, cuda), W, a2, a1,
+                                     a_t, a_n)
+    sdk.sd_device_status()
+    rx, rd = oracle.cfg_dpmpp_3m_step(x, eu, ec, d1, d2, W, a2, a1, a_t, a_n)
+    assert rel_err(xo.cpu().numpy(), rx) <= REL_STEP
+    assert rel_err(d.cpu().numpy(), rd) <= REL_STEP
+
+
+def test_third_order_twenty_step_run(cuda):
+    # serving latent, Karras sigmas, orders 1, 2, 3, ..., 3, 1; history rotated through three buffers
+    shape = si.WORKLOADS[5].latent
+    sched = sdk.dpmpp_3m_schedule(20)
+    x0 = si.normal(shape, 1800)
+    eps = [(si.normal(shape, 1900 + 2 * i), si.normal(shape, 1901 + 2 * i)) for i in range(20)]
+    xd = _t(x0, cuda)
+    bufs = [torch.zeros(shape, device=cuda) for _ in range(3)]
+    for i, ((a2, a1, a_t, a_n, order), (eu, ec)) in enumerate(zip(sched, eps)):
+        d_out, d1, d2 = bufs[i % 3], bufs[(i - 1) % 3], bufs[(i - 2) % 3]
+        if order == 3:
+            sdk.sd_cfg_dpmpp_3m_step(xd, _t(eu, cuda), _t(ec, cuda), d1, d2, W, a2, a1, a_t, a_n, out=xd, d_out=d_out)
+        else:
+            sdk.sd_cfg_dpmpp_2m_step(xd, _t(eu, cuda), _t(ec, cuda), d1, W, a1, a_t, a_n, order, out=xd, d_out=d_out)
+    sdk.sd_device_status()
+    ref = oracle.cfg_dpmpp_3m_loop(x0, eps, W, oracle.dpmpp_3m_schedule(20))
+    assert rel_err(xd.cpu().numpy(), ref) <= REL_LOOP

@@ -166,3 +166,24 @@ def test_third_order_reproduces_a_linear_data_prediction_exactly_up_to_the_warm_
     F = lambda u: np.exp(u) * (0.3 + 0.8 * (u - 1))
     exact = sig(ls[3]) / sig(ls[2]) * x + sig(ls[3]) * (F(ls[3]) - F(ls[2]))
     np.testing.assert_allclose(xn, exact, rtol=1e-12)
+
+
+def test_third_order_schedule_and_loop_end_on_the_data():
+    sched = oracle.dpmpp_3m_schedule(20)
+    assert [o for *_, o in sched] == [1, 2] + [3] * 17 + [1] and sched[-1][3] == 1.0
+    x0 = normal((256,), 9).astype(np.float64)
+    a0 = sched[0][2]
+    x = np.sqrt(a0) * x0 + np.sqrt(1 - a0) * normal((256,), 10).astype(np.float64)
+    eps = []
+    # noise predictions consistent with the constant data prediction x0 along the run
+    xs, hist = x.copy(), []
+    for a_p2, a_p1, a_t, a_n, order in sched:
+        g = (xs - np.sqrt(a_t) * x0) / np.sqrt(1 - a_t)
+        eps.append((g, g))
+        if order == 3:
+            xs, d = oracle.dpmpp_3m_step(xs, g, hist[-1], hist[-2], a_p2, a_p1, a_t, a_n)
+        else:
+            xs, d = oracle.dpmpp_2m_step(xs, g, hist[-1] if hist else None, a_p1, a_t, a_n, order)
+        hist.append(d)
+    np.testing.assert_allclose(xs, x0, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(oracle.cfg_dpmpp_3m_loop(x, eps, 7.5, sched), x0, rtol=1e-10, atol=1e-10)

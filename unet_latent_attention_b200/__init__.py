@@ -18,7 +18,8 @@ import math
 import os
 import re
 
-from .schedule import ddim_schedule, dpmpp_2m_schedule, karras_alpha_bars, scaled_linear_alphas_cumprod  # noqa: F401
+from .schedule import (ddim_schedule, dpmpp_2m_schedule, dpmpp_3m_schedule, karras_alpha_bars,  # noqa: F401
+                       scaled_linear_alphas_cumprod)
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libsdk.so")
@@ -56,13 +57,14 @@ def lib() -> ctypes.CDLL:
         L.sd_attention_layout.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, i64, f32, c_int, c_int, vp]
         L.sd_cfg_ddim_step.argtypes = [vp, vp, vp, vp, i64, f32, f64, f64, vp]
         L.sd_cfg_dpmpp_2m_step.argtypes = [vp, vp, vp, vp, vp, vp, i64, f32, f64, f64, f64, c_int, vp]
+        L.sd_cfg_dpmpp_3m_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, f32, f64, f64, f64, f64, vp]
         L.sd_device_status.argtypes = [vp, c_int]
         L.sd_debug_set_fault.argtypes = [c_int]
         L.sd_debug_set_fault.restype = None
         for f in ("sd_group_norm", "sd_group_norm_silu", "sd_attention", "sd_attention_noalloc", "sd_attention_f16",
                   "sd_attention_layout",
                   "sd_cfg_ddim_step",
-                  "sd_cfg_dpmpp_2m_step", "sd_device_status"):
+                  "sd_cfg_dpmpp_2m_step", "sd_cfg_dpmpp_3m_step", "sd_device_status"):
             getattr(L, f).restype = c_int
         L.sd_status_string.argtypes = [c_int]
         L.sd_status_string.restype = ctypes.c_char_p
@@ -238,6 +240,23 @@ def sd_cfg_dpmpp_2m_step(x, eps_u, eps_c, d_prev, w: float, alpha_prev: float, a
     _check("sd_cfg_dpmpp_2m_step", lib().sd_cfg_dpmpp_2m_step(
         x.data_ptr(), eps_u.data_ptr(), eps_c.data_ptr(), d_prev.data_ptr() if d_prev is not None else None,
         out.data_ptr(), d_out.data_ptr(), x.numel(), w, alpha_prev, alpha_t, alpha_next, int(order), _stream(x)))
+    return out, d_out
+
+
+def sd_cfg_dpmpp_3m_step(x, eps_u, eps_c, d_prev, d_prev2, w: float, alpha_prev2: float, alpha_prev: float,
+                         alpha_t: float, alpha_next: float, out=None, d_out=None):
+    """Guided third-order multistep DPM-Solver++ step; returns (x_next, d). ``out`` may be ``x``;
+    ``d_out`` may be ``d_prev`` or ``d_prev2``."""
+    import torch
+    for t in (x, eps_u, eps_c, d_prev, d_prev2):
+        if t.dtype != torch.float32 or t.shape != x.shape:
+            raise ValueError("sd_cfg_dpmpp_3m_step takes fp32 tensors of one shape")
+    out = torch.empty_like(x) if out is None else out
+    d_out = torch.empty_like(x) if d_out is None else d_out
+    _require_cuda(x, eps_u, eps_c, d_prev, d_prev2, out, d_out)
+    _check("sd_cfg_dpmpp_3m_step", lib().sd_cfg_dpmpp_3m_step(
+        x.data_ptr(), eps_u.data_ptr(), eps_c.data_ptr(), d_prev.data_ptr(), d_prev2.data_ptr(), out.data_ptr(),
+        d_out.data_ptr(), x.numel(), w, alpha_prev2, alpha_prev, alpha_t, alpha_next, _stream(x)))
     return out, d_out
 
 

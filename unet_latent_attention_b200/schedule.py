@@ -46,3 +46,14 @@ def dpmpp_2m_schedule(steps: int = 20):
     """[(alpha_prev, alpha_t, alpha_next, order)] for sd_cfg_dpmpp_2m_step over a whole sampling run."""
     ab = karras_alpha_bars(steps) + [1.0]
     return [(ab[i - 1] if i else ab[0], ab[i], ab[i + 1], 1 if i in (0, steps - 1) else 2) for i in range(steps)]
+
+
+def dpmpp_3m_schedule(steps: int = 20):
+    """[(alpha_prev2, alpha_prev, alpha_t, alpha_next, order)] for a third-order run: order 1, then 2,
+    then 3, with the last step (to sigma = 0) first order. Unused history slots repeat alpha_t."""
+    ab = karras_alpha_bars(steps) + [1.0]
+    out = []
+    for i in range(steps):
+        order = 1 if i in (0, steps - 1) else min(i + 1, 3)
+        out.append((ab[i - 2] if i >= 2 else ab[i], ab[i - 1] if i >= 1 else ab[i], ab[i], ab[i + 1], order))
+    return out
