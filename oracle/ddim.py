@@ -11,7 +11,7 @@ Sampler step: the engine page §1 names the update step(z_t, noise_pred, t) as D
 with eta = 0 on the cumulative products alpha_bar,
     x0_hat = (x - sqrt(1 - alpha_t) g) / sqrt(alpha_t)
     x'     = sqrt(alpha_prev) x0_hat + sqrt(1 - alpha_prev) g
-with no clipping of x0_hat. Schedule for the multi-step driver (not printed either): the
+with no clipping of x0_hat. Schedule for the multi-step sampling loop (not printed either): the
 Stable Diffusion "scaled linear" betas, beta_i = linspace(sqrt(0.00085), sqrt(0.012), 1000)_i^2,
 alpha_bar_t = prod_{i<=t} (1 - beta_i), timesteps 950, 900, ..., 0 and alpha_prev = 1 after the
 last step.
@@ -58,7 +58,7 @@ def ddim_timesteps(T: int = 1000, steps: int = 20) -> np.ndarray:
 
 
 def ddim_schedule(steps: int = 20, T: int = 1000, beta_start: float = 0.00085, beta_end: float = 0.012):
-    """List of (t, alpha_t, alpha_prev) for the driver; alpha_prev = 1 after the final step."""
+    """List of (t, alpha_t, alpha_prev) for the sampling loop; alpha_prev = 1 after the final step."""
     ac = alphas_cumprod(scaled_linear_betas(beta_start, beta_end, T))
     ts = ddim_timesteps(T, steps)
     out = []

@@ -54,7 +54,7 @@ def test_scaled_linear_schedule_definition():
     assert (np.diff(ac) < 0).all() and 0.004 < ac[-1] < 0.006
 
 
-def test_timesteps_and_driver_schedule():
+def test_timesteps_and_loop_schedule():
     ts = oracle.ddim_timesteps(1000, 20)
     assert list(ts) == list(range(950, -1, -50))
     sched = oracle.ddim_schedule(20)
