@@ -230,6 +230,14 @@ const char* sd_last_error(void);
 sd_status sd_device_status(void* stream, int reset);
 
 /*
+ * Test hook, pure host code: writes to out[0 .. grid] the unit boundaries that sd_attention's
+ * persistent grid uses for `items` query-tile items of `nkv` K/V tiles on `grid` CTAs (CTA c owns
+ * units [out[c], out[c+1])), with the schedule cost model of head dim `dh`. SD_ERR_INVALID_ARG if
+ * items, nkv or grid is < 1, grid > 256, grid > items, or out is NULL.
+ */
+sd_status sd_debug_attention_ranges(int64_t items, int64_t nkv, int64_t grid, int64_t dh, int64_t* out);
+
+/*
  * Test hook for the failure path: flags bit 0 makes every later sd_attention launch (any thread,
  * any device) skip loading its first V tile, so each CTA's bounded wait expires after about one
  * second, the CTA drains its own copies, frees its tensor memory and returns, and

@@ -142,3 +142,49 @@ def test_schedule_tables_match_the_oracle():
     assert [t for t, _, _ in ours] == [t for t, _, _ in ref]
     for (_, a, p), (_, ra, rp) in zip(ours, ref):
         assert abs(a - ra) < 1e-13 and abs(p - rp) < 1e-13
+
+
+def _ranges(L, items, nkv, grid, dh):
+    import ctypes
+    L.sd_debug_attention_ranges.argtypes = [ctypes.c_int64] * 4 + [ctypes.POINTER(ctypes.c_int64)]
+    L.sd_debug_attention_ranges.restype = ctypes.c_int
+    out = (ctypes.c_int64 * (grid + 1))()
+    assert L.sd_debug_attention_ranges(items, nkv, grid, dh, out) == 0
+    return list(out)
+
+
+def _cost(a, b, nkv, m):
+    segs = (b - 1) // nkv - a // nkv + 1
+    return (b - a) + m[0] * (segs - 1) + (m[1] if a % nkv else 0) + (m[2] if b % nkv else 0)
+
+
+@pytest.mark.parametrize("items,nkv,grid,dh", [(256, 32, 148, 40), (320, 32, 148, 64), (576, 72, 148, 40),
+                                                (160, 5, 148, 40), (240, 5, 148, 80), (256, 1, 148, 40),
+                                                (149, 3, 148, 160), (1000, 17, 132, 40)])
+def test_persistent_grid_ranges(L, items, nkv, grid, dh):
+    # host logic of the attention schedule: contiguous cover of all units, no range strictly inside
+    # one item (an item spans at most two consecutive CTAs), empty ranges only at the end, and a
+    # largest modelled cost no worse than equal unit counts
+    u = _ranges(L, items, nkv, grid, dh)
+    U = items * nkv
+    assert u[0] == 0 and u[-1] == U and all(a <= b for a, b in zip(u, u[1:]))
+    for a, b in zip(u, u[1:]):
+        if b > a:
+            assert not (a % nkv and b % nkv and a // nkv == (b - 1) // nkv), (a, b)
+    nonempty = [b > a for a, b in zip(u, u[1:])]
+    assert nonempty == sorted(nonempty, reverse=True)
+    if nkv == 1:
+        assert u == [U * c // grid for c in range(grid + 1)]
+    else:
+        m = (1.3, 0.5, 1.4) if dh == 64 else (1.0, 0.6, 0.9)
+        worst = max(_cost(a, b, nkv, m) for a, b in zip(u, u[1:]) if b > a)
+        even = max(_cost(U * c // grid, U * (c + 1) // grid, nkv, m) for c in range(grid))
+        assert worst <= even + 1e-9
+
+
+def test_persistent_grid_ranges_rejects_bad_arguments(L):
+    import ctypes
+    out = (ctypes.c_int64 * 300)()
+    L.sd_debug_attention_ranges.argtypes = [ctypes.c_int64] * 4 + [ctypes.POINTER(ctypes.c_int64)]
+    assert L.sd_debug_attention_ranges(10, 4, 20, 40, out) == 1  # grid > items
+    assert L.sd_debug_attention_ranges(1000, 4, 257, 40, out) == 1  # grid > 256

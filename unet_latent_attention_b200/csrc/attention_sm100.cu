@@ -1235,6 +1235,18 @@ extern "C" sd_status sd_attention_noalloc(const void* q, const void* k, const vo
   return attention_impl(q, k, v, o, B, heads, Lq, Lk, dh, scale, stream, true);
 }
 
+// Test hook (declared in sd_kernels.h): the unit ranges the persistent grid would use for `items`
+// items of `nkv` K/V tiles on `grid` CTAs with the cost model of head dim `dh`; pure host code.
+extern "C" sd_status sd_debug_attention_ranges(int64_t items, int64_t nkv, int64_t grid, int64_t dh, int64_t* out) {
+  if (items < 1 || nkv < 1 || grid < 1 || grid > kMaxCtas || grid > items || !out)
+    return sd::fail(SD_ERR_INVALID_ARG, "sd_debug_attention_ranges: bad arguments");
+  const CostModel m = dh == 64 ? CostModel{1.3, 0.5, 1.4} : CostModel{1.0, 0.6, 0.9};
+  long long u[kMaxCtas + 1];
+  part_ranges(items * nkv, nkv, static_cast<int>(grid), m, u);
+  for (int64_t c = 0; c <= grid; ++c) out[c] = u[c];
+  return SD_OK;
+}
+
 // Test hook (declared in sd_kernels.h): bit 0 makes the next attention launches skip their first
 // V tile so that the kernel's bounded wait expires and reports SD_ERR_TIMEOUT.
 extern "C" void sd_debug_set_fault(int flags) { g_debug_flags = flags; }
