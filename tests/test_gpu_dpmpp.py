@@ -109,3 +109,14 @@ def test_third_order_twenty_step_run(cuda):
     sdk.sd_device_status()
     ref = oracle.cfg_dpmpp_3m_loop(x0, eps, W, oracle.dpmpp_3m_schedule(20))
     assert rel_err(xd.cpu().numpy(), ref) <= REL_LOOP
+
+
+def test_third_order_in_place_over_the_oldest_history(cuda):
+    # d_out may overwrite d_prev2 (the history rotates through two buffers), x_out may be x
+    x, eu, ec, d1 = _inputs((70001,), 2000)
+    d2 = si.normal((70001,), 2010)
+    xd, d1d, d2d = _t(x, cuda), _t(d1, cuda), _t(d2, cuda)
+    sdk.sd_cfg_dpmpp_3m_step(xd, _t(eu, cuda), _t(ec, cuda), d1d, d2d, W, 0.2, 0.25, 0.3, 0.4, out=xd, d_out=d2d)
+    sdk.sd_device_status()
+    rx, rd = oracle.cfg_dpmpp_3m_step(x, eu, ec, d1, d2, W, 0.2, 0.25, 0.3, 0.4)
+    assert rel_err(xd.cpu().numpy(), rx) <= REL_STEP and rel_err(d2d.cpu().numpy(), rd) <= REL_STEP

@@ -59,3 +59,12 @@ def test_unaligned_view_takes_streaming_path(cuda):
     y = sdk.sd_group_norm(x, gamma, beta, 32, 1e-5)
     ref = oracle.group_norm(x.cpu().numpy(), np.ones(64), np.zeros(64), 32, 1e-5)
     assert rel_err(y.cpu().numpy(), ref) <= REL
+
+
+@pytest.mark.parametrize("B", [2, 3])
+def test_sdxl_top_level_groups(cuda, B):
+    # 10 x 16384-element groups: 512-thread CTAs with 10 float4 per thread, two per SM
+    shape = si.GNShape(B, 320, 128, 128)
+    x, gamma, beta = si.group_norm_inputs(4, shape, sub=11 + B)
+    y = _gn(x, gamma, beta, 32, 1e-5, cuda)
+    assert rel_err(y, oracle.group_norm(x, gamma, beta, 32, 1e-5)) <= REL

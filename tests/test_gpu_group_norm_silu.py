@@ -69,3 +69,11 @@ def test_bf16_output_may_not_overlap_x(cuda):
     y = x.view(torch.bfloat16).reshape(-1)[:x.numel()].view(x.shape)  # x's first bytes as bf16
     with pytest.raises(sdk.SDError):
         sdk.sd_group_norm_silu(x, torch.ones(64, device=cuda), torch.zeros(64, device=cuda), 32, 1e-5, out=y)
+
+
+@pytest.mark.parametrize("bf16", [False, True], ids=["f32", "bf16"])
+def test_sdxl_top_level_groups(cuda, bf16):
+    shape = si.GNShape(2, 320, 128, 128)
+    x, gamma, beta = si.group_norm_inputs(4, shape, sub=21)
+    y = _run(x, gamma, beta, 32, 1e-5, cuda, bf16)
+    _check(y, oracle.group_norm_silu(x, gamma, beta, 32, 1e-5), bf16)
