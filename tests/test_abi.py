@@ -188,3 +188,21 @@ def test_persistent_grid_ranges_rejects_bad_arguments(L):
     L.sd_debug_attention_ranges.argtypes = [ctypes.c_int64] * 4 + [ctypes.POINTER(ctypes.c_int64)]
     assert L.sd_debug_attention_ranges(10, 4, 20, 40, out) == 1  # grid > items
     assert L.sd_debug_attention_ranges(1000, 4, 257, 40, out) == 1  # grid > 256
+
+
+def test_binding_argument_checks_on_the_host():
+    # checks the bindings make before any device work (CPU tensors suffice to reach them)
+    q16 = torch.zeros(1, 1, 8, 40, dtype=torch.float16)
+    with pytest.raises(ValueError, match="all bf16 or all fp16"):
+        sdk.sd_attention(q16, q16.to(torch.bfloat16), q16)
+    with pytest.raises(ValueError, match="layout"):
+        sdk.sd_attention(q16, q16, q16, layout="lbhd")
+    with pytest.raises(ValueError, match="fp32"):
+        sdk.sd_group_norm_silu(torch.zeros(1, 32, 4, 4, dtype=torch.float64), torch.ones(32), torch.zeros(32))
+    x = torch.zeros(16)
+    with pytest.raises(ValueError, match="order 2 needs d_prev"):
+        sdk.sd_cfg_dpmpp_2m_step(x, x, x, None, 7.5, 0.2, 0.3, 0.4, 2)
+    with pytest.raises(ValueError, match="one shape"):
+        sdk.sd_cfg_dpmpp_3m_step(x, x, x, x, torch.zeros(8), 7.5, 0.1, 0.2, 0.3, 0.4)
+    with pytest.raises(ValueError, match="CUDA"):
+        sdk.sd_cfg_dpmpp_2m_step(x, x, x, None, 7.5, 0.2, 0.3, 0.4, 1)
