@@ -225,7 +225,9 @@ const char* sd_last_error(void);
 /*
  * Synchronises `stream`, then reads the current device's status word. Returns SD_ERR_TIMEOUT if
  * any kernel of this library gave up a bounded wait since the last reset, SD_ERR_CUDA if the
- * synchronisation failed, SD_OK otherwise. reset != 0 clears the word afterwards.
+ * synchronisation failed, SD_OK otherwise. reset != 0 clears the word afterwards; if a kernel had
+ * given up, it also clears sd_attention's hand-off workspace on this device (an aborted launch may
+ * have left split-item flags set).
  */
 sd_status sd_device_status(void* stream, int reset);
 
