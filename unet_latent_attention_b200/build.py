@@ -6,6 +6,7 @@ Run ``python -m unet_latent_attention_b200.build`` (or ``__graft_entry__.build()
 from __future__ import annotations
 
 import concurrent.futures as cf
+import fcntl
 import os
 import shutil
 import subprocess
@@ -64,22 +65,32 @@ def build(verbose_ptxas: bool = False, force: bool = False, defines=(), out: str
     return _build(verbose_ptxas, force, [], lib_path)
 
 
-def _build(verbose_ptxas: bool, force: bool, extra, lib_path: str) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def _up_to_date(lib_path: str) -> bool:
     srcs = sources()
     deps = srcs + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
     deps.append(os.path.join(INCLUDE, "sd_kernels.h"))
-    if (not force and not verbose_ptxas and os.path.exists(lib_path)
-            and os.path.getmtime(lib_path) >= max(os.path.getmtime(d) for d in deps)):
+    return os.path.exists(lib_path) and os.path.getmtime(lib_path) >= max(os.path.getmtime(d) for d in deps)
+
+
+def _build(verbose_ptxas: bool, force: bool, extra, lib_path: str) -> str:
+    os.makedirs(BUILD, exist_ok=True)
+    if not force and not verbose_ptxas and _up_to_date(lib_path):
         return lib_path
-    with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas, extra), srcs))
-    tmp = lib_path + ".tmp"
-    cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lpthread", "-lrt"]
-    r = subprocess.run(cmd, capture_output=True, text=True)
-    if r.returncode != 0:
-        raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, lib_path)
+    # Concurrent callers (one process per GPU, parallel test workers) build one at a time; whoever
+    # gets the lock second finds the library fresh and returns.
+    with open(os.path.join(BUILD, ".lock"), "w") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        if not force and not verbose_ptxas and _up_to_date(lib_path):
+            return lib_path
+        srcs = sources()
+        with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
+            objs = list(ex.map(lambda s: _compile(s, verbose_ptxas, extra), srcs))
+        tmp = f"{lib_path}.{os.getpid()}.tmp"
+        cmd = [nvcc(), *ARCH, "-shared", "-o", tmp, *objs, "-lcudart_static", "-ldl", "-lpthread", "-lrt"]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        if r.returncode != 0:
+            raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
+        os.replace(tmp, lib_path)
     return lib_path
 
 
