@@ -187,3 +187,109 @@ def test_third_order_schedule_and_loop_end_on_the_data():
         hist.append(d)
     np.testing.assert_allclose(xs, x0, rtol=1e-10, atol=1e-10)
     np.testing.assert_allclose(oracle.cfg_dpmpp_3m_loop(x, eps, 7.5, sched), x0, rtol=1e-10, atol=1e-10)
+
+
+# ---- guidance wiring and history bookkeeping of the guided steps and loops
+#
+# The guided steps combine the two noise predictions as eps_u + w (eps_c - eps_u) (the CFG loop of
+# the engine page §7 and the deployment page's 示例说明) before the solver step. With w != 1 and
+# eps_u != eps_c, the pins below build the pair so that only the correct combination gives the noise
+# prediction g consistent with a known data prediction; swapping the pair gives g + a (2 - 1/w).
+
+W = 7.5
+
+
+def _guided_pair(g, seed):
+    """(eps_u, eps_c) with eps_u + W (eps_c - eps_u) = g and eps_u != eps_c."""
+    a = normal(np.shape(g), seed).astype(np.float64)
+    return g + a, g + a * (1.0 - 1.0 / W)
+
+
+def test_guided_pair_construction():
+    g = normal((64,), 20).astype(np.float64)
+    eu, ec = _guided_pair(g, 21)
+    np.testing.assert_allclose(oracle.cfg(eu, ec, W), g, rtol=0, atol=1e-12)
+    assert np.abs(oracle.cfg(ec, eu, W) - g).max() > 0.5  # the swapped order is far off
+
+
+@pytest.mark.parametrize("order", [1, 2])
+def test_guided_2m_step_lands_on_the_closed_form(order):
+    # constant data prediction x0: the exponential integrator is exact for both orders
+    x0, e = normal((512,), 22).astype(np.float64), normal((512,), 23).astype(np.float64)
+    a_p, a_t, a_n = 0.1, 0.2, 0.45
+    x = np.sqrt(a_t) * x0 + np.sqrt(1 - a_t) * e
+    g = (x - np.sqrt(a_t) * x0) / np.sqrt(1 - a_t)
+    eu, ec = _guided_pair(g, 24)
+    xn, D = oracle.cfg_dpmpp_2m_step(x, eu, ec, x0, W, a_p, a_t, a_n, order)
+    np.testing.assert_allclose(D, x0, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(xn, np.sqrt(a_n) * x0 + np.sqrt(1 - a_n) * e, rtol=1e-12, atol=1e-12)
+
+
+def test_guided_3m_step_lands_on_the_closed_form():
+    x0, e = normal((512,), 25).astype(np.float64), normal((512,), 26).astype(np.float64)
+    a2, a1, a_t, a_n = 0.05, 0.1, 0.2, 0.45
+    x = np.sqrt(a_t) * x0 + np.sqrt(1 - a_t) * e
+    g = (x - np.sqrt(a_t) * x0) / np.sqrt(1 - a_t)
+    eu, ec = _guided_pair(g, 27)
+    xn, D = oracle.cfg_dpmpp_3m_step(x, eu, ec, x0, x0, W, a2, a1, a_t, a_n)
+    np.testing.assert_allclose(D, x0, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(xn, np.sqrt(a_n) * x0 + np.sqrt(1 - a_n) * e, rtol=1e-12, atol=1e-12)
+
+
+def _lam_of(ab):
+    return 0.5 * np.log(ab / (1.0 - ab))
+
+
+def _sig(ab):
+    return np.sqrt(1.0 - ab)
+
+
+def _run_guided(loop, x, sched, D_of_lambda, seed):
+    """Drives `loop` with guided noise pairs that, at each step's state, are consistent with the data
+    prediction D(lambda_t). The states come from the loop itself run on growing prefixes of the
+    schedule (every prefix run starts from the same x); returns the full run's result and the pairs."""
+    eps = []
+    xs = np.array(x, np.float64)
+    for i, row in enumerate(sched):
+        a_t = row[1] if len(row) == 4 else row[2]  # (a_p, a_t, a_n, order) or (a_p2, a_p1, a_t, a_n, order)
+        g = (xs - np.sqrt(a_t) * D_of_lambda(_lam_of(a_t))) / np.sqrt(1 - a_t)
+        eps.append(_guided_pair(g, seed + i))
+        xs = loop(x, eps, W, sched[: i + 1])
+    return xs, eps
+
+
+def test_guided_2m_loop_is_the_midpoint_exponential_integrator_on_a_linear_data_prediction():
+    # For D(lambda) = c0 + c1 lambda, the second-order combination (1 + 1/(2r)) D_t - D_prev / (2r)
+    # equals D at the midpoint lambda_t + h/2 exactly, so each order-2 step of a correct loop is
+    #   x' = (sigma'/sigma) x + sigma' (e^lambda' - e^lambda) D(lambda + h/2),
+    # and an order-1 step uses D(lambda). This needs D_prev and alpha_prev of the PREVIOUS step.
+    c0, c1 = 0.4, -0.9
+    D = lambda l: c0 + c1 * l
+    sched = oracle.dpmpp_2m_schedule(12)[:-1]  # stop before the step to sigma = 0 (it returns D alone)
+    x = normal((8,), 28).astype(np.float64)
+    got, _ = _run_guided(oracle.cfg_dpmpp_2m_loop, x, sched, D, 300)
+    ref = x.copy()
+    for a_p, a_t, a_n, order in sched:
+        l_t, l_n = _lam_of(a_t), _lam_of(a_n)
+        l_mid = l_t if order == 1 else l_t + 0.5 * (l_n - l_t)
+        ref = _sig(a_n) / _sig(a_t) * ref + _sig(a_n) * (np.exp(l_n) - np.exp(l_t)) * D(l_mid)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_guided_3m_loop_is_exact_after_its_warm_up_on_a_quadratic_data_prediction():
+    # Orders 1 and 2 open the run; from the third step on, each order-3 step integrates
+    # e^lambda D(lambda) exactly when D is quadratic and the two history entries are the data
+    # predictions of the previous two steps, newest first. The exact flow is affine in x, so the
+    # loop's result must equal (sigma_K / sigma_2) x_2 + sigma_K (F(lambda_K) - F(lambda_2)), where
+    # x_2 is the state after the two warm-up steps and F' = e^u D(u).
+    c = (0.7, -1.3, 0.9)
+    D = lambda l: c[0] + c[1] * l + c[2] * l * l
+    F = lambda u: np.exp(u) * (c[0] + c[1] * (u - 1) + c[2] * (u * u - 2 * u + 2))
+    sched = oracle.dpmpp_3m_schedule(14)[:-1]
+    assert [o for *_, o in sched] == [1, 2] + [3] * 11
+    x = normal((8,), 29).astype(np.float64)
+    got, eps = _run_guided(oracle.cfg_dpmpp_3m_loop, x, sched, D, 400)
+    x2 = oracle.cfg_dpmpp_3m_loop(x, eps[:2], W, sched[:2])
+    a2, aK = sched[2][2], sched[-1][3]
+    ref = _sig(aK) / _sig(a2) * x2 + _sig(aK) * (F(_lam_of(aK)) - F(_lam_of(a2)))
+    np.testing.assert_allclose(got, ref, rtol=1e-10, atol=1e-11)
