@@ -97,6 +97,12 @@ sd_status sd_group_norm_silu(const float* x, const float* gamma, const float* be
  *  scale  : finite; callers normally pass 1/sqrt(dh).
  *  Lq, Lk : >= 1 and <= 2^30, any value (ragged tails are masked). B*heads < 2^31.
  * All four pointers must be 16-byte aligned (SD_ERR_MISALIGNED otherwise).
+ * Scratch: when a shape has more query-tile items than the GPU has SMs, some items are split
+ * between two CTAs of the persistent grid, which hand partial results over through a per-device
+ * workspace that the first such call allocates (cudaMalloc, about 50-100 KB per SM) and later calls
+ * grow; sd_attention_noalloc avoids that allocation. The hand-off never waits for a CTA to be
+ * scheduled, so the launch needs no particular number of free SMs; two launches that split items
+ * must not run concurrently on one device (they share the workspace).
  */
 sd_status sd_attention(const void* q, const void* k, const void* v, void* o,
                        int64_t B, int64_t heads, int64_t Lq, int64_t Lk, int64_t dh, float scale,
@@ -142,8 +148,10 @@ sd_status sd_attention_layout(const void* q, const void* k, const void* v, void*
  * to 148 SMs). A shape whose scratch would exceed 16 MiB is rejected with SD_ERR_UNSUPPORTED and
  * nothing is launched.
  *
- *  - The first call on a device looks up the array's device address (cudaGetSymbolAddress); make
- *    that first call before any stream capture on that device.
+ *  - Every call first looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress, cached per device and CUDA context, so a context created again after
+ *    cudaDeviceReset is noticed); the first call on a device does the actual lookup, so make that
+ *    first call before any stream capture on that device.
  *  - Every call uses the same array, which keeps the previous call's contents; each call clears
  *    the part that must start at zero with an asynchronous memset on `stream` before its kernel.
  *  - Calls whose executions overlap on the GPU (different streams, no ordering between them) race
@@ -243,8 +251,10 @@ sd_status sd_debug_attention_ranges(int64_t items, int64_t nkv, int64_t grid, in
  * Test hook for the failure path: flags bit 0 makes every later sd_attention launch (any thread,
  * any device) skip loading its first V tile, so each CTA's bounded wait expires after about one
  * second, the CTA drains its own copies, frees its tensor memory and returns, and
- * sd_device_status() reports SD_ERR_TIMEOUT. Outputs of such launches are undefined. flags = 0
- * restores normal operation. Not for production use.
+ * sd_device_status() reports SD_ERR_TIMEOUT. Outputs of such launches are undefined. Bit 1 holds
+ * back the tail piece of every item split between two CTAs by about 50 us, so that the head piece
+ * finishes first and the tail piece merges (the results are unchanged). flags = 0 restores normal
+ * operation. Not for production use.
  */
 void sd_debug_set_fault(int flags);
 

@@ -206,3 +206,23 @@ def test_binding_argument_checks_on_the_host():
         sdk.sd_cfg_dpmpp_3m_step(x, x, x, x, torch.zeros(8), 7.5, 0.1, 0.2, 0.3, 0.4)
     with pytest.raises(ValueError, match="CUDA"):
         sdk.sd_cfg_dpmpp_2m_step(x, x, x, None, 7.5, 0.2, 0.3, 0.4, 1)
+
+
+def test_noalloc_binding_checks_type_and_shapes_on_the_host():
+    # an fp16 tensor or mismatched k/v must never reach the bf16 kernel
+    q = torch.zeros(1, 2, 8, 40, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="bf16"):
+        sdk.sd_attention_noalloc(q.to(torch.float16), q.to(torch.float16), q.to(torch.float16))
+    with pytest.raises(ValueError, match="bf16"):
+        sdk.sd_attention_noalloc(q, q, q.to(torch.float16))
+    with pytest.raises(ValueError, match="matching q"):
+        sdk.sd_attention_noalloc(q, torch.zeros(1, 2, 9, 40, dtype=torch.bfloat16), q)
+    with pytest.raises(ValueError, match="matching q"):
+        sdk.sd_attention_noalloc(q, torch.zeros(1, 3, 8, 40, dtype=torch.bfloat16),
+                                 torch.zeros(1, 3, 8, 40, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="4-D"):
+        sdk.sd_attention_noalloc(q[0], q, q)
+    with pytest.raises(ValueError, match="out"):
+        sdk.sd_attention_noalloc(q, q, q, out=torch.zeros(1, 2, 8, 40, dtype=torch.float32))
+    with pytest.raises(ValueError, match="CUDA"):
+        sdk.sd_attention_noalloc(q, q, q)

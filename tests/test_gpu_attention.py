@@ -111,6 +111,25 @@ def test_split_items_persistent_schedule(cuda, dh, heads, Lq, Lk):
     _check(o, oracle.attention(q, k, v))
 
 
+@pytest.mark.parametrize("dh,heads,Lq,Lk", [(40, 80, 256, 640), (64, 80, 256, 1000), (80, 80, 256, 700),
+                                            (160, 120, 128, 300)])
+def test_split_items_either_piece_may_merge(cuda, dh, heads, Lq, Lk):
+    # test hook bit 1 holds the tail pieces back, so the head pieces publish and the tail pieces
+    # merge: the output must be bit-identical to the usual order (one fixed merge order)
+    q, k, v = _qkv(2, heads, Lq, Lk, dh, 9200 + dh + Lk)
+    qd, kd, vd = q.to(cuda), k.to(cuda), v.to(cuda)
+    usual = sdk.sd_attention(qd, kd, vd)
+    sdk.sd_device_status()
+    try:
+        sdk.sd_debug_set_fault(2)
+        reversed_ = sdk.sd_attention(qd, kd, vd)
+        sdk.sd_device_status()
+    finally:
+        sdk.sd_debug_set_fault(0)
+    assert torch.equal(usual, reversed_)
+    _check(reversed_.float().cpu().numpy(), oracle.attention(q, k, v))
+
+
 def test_repeated_launches_reuse_the_hand_off_flags(cuda):
     # the split hand-off flags must return to zero after every launch (graph replays rely on it)
     q, k, v = _qkv(2, 80, 256, 640, 40, 9100)

@@ -180,7 +180,8 @@ def sd_attention(q, k, v, scale: float | None = None, out=None, layout: str = "b
 
 
 def sd_attention_noalloc(q, k, v, scale: float | None = None, out=None):
-    """sd_attention without any device allocation by the library (fixed 16 MiB scratch instead).
+    """sd_attention (bf16, [B, heads, L, dh]) without any device allocation by the library: its
+    split-item scratch is a fixed 16 MiB device array instead of a cudaMalloc'd workspace.
 
     For callers that cannot let a library call cudaMalloc: inside CUDA-graph capture, under a
     framework that owns all device memory, or in loops that cannot absorb cudaMalloc's implicit
@@ -188,14 +189,23 @@ def sd_attention_noalloc(q, k, v, scale: float | None = None, out=None):
     overlap on the GPU race on the shared scratch.
     """
     import torch
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise ValueError("sd_attention_noalloc takes bf16 q, k, v")
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, heads, L, dh]")
+    B, Hh, Lq, dh = q.shape
+    Lk = k.shape[2]
+    if k.shape != (B, Hh, Lk, dh) or v.shape != k.shape:
+        raise ValueError("k and v must be [B, heads, Lk, dh] matching q")
     if out is None:
         out = torch.empty_like(q)
+    if out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must have the shape and type of q")
     _require_cuda(q, k, v, out)
-    B, Hh, Lq, dh = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(dh)
     _check("sd_attention_noalloc", lib().sd_attention_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                                              out.data_ptr(), B, Hh, Lq, k.shape[2], dh, scale,
+                                                              out.data_ptr(), B, Hh, Lq, Lk, dh, scale,
                                                               _stream(q)))
     return out
 

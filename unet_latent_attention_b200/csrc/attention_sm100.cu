@@ -50,69 +50,6 @@ using namespace sm100;
 #define SD_POLY_PAIRS -1  // tuning override of the per-head-dim choice in the launch table
 #endif
 
-#ifdef SD_TRACE
-// Tuning builds only: per-CTA phase timestamps of the first softmax warp and of the MMA warp.
-constexpr int kTraceCtas = 64, kTraceIters = 40, kTraceSlots = 8, kTraceLast = kTraceIters - 1;
-__device__ long long g_trace[kTraceCtas][12][kTraceIters][kTraceSlots];
-__device__ unsigned long long g_span[1024][2];  // global-timer ns at CTA entry and exit
-__device__ unsigned long long g_span_seq[8][1024][2];  // the same per launch (launch index mod 8)
-__device__ unsigned int g_span_entries;
-__device__ unsigned int g_span_smid[1024];
-__device__ unsigned long long g_seg[1024][8];  // release of the grid dependency, then segment ends
-#define SD_SEG(slot)                                                                          \
-  do {                                                                                        \
-    if (blockIdx.x < 1024 && (slot) < 8) g_seg[blockIdx.x][slot] = gtimer();                  \
-  } while (0)
-__device__ __forceinline__ unsigned long long gtimer() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-#define SD_SPAN(slot)                                                                \
-  do {                                                                               \
-    if (threadIdx.x == 0 && blockIdx.x < 1024) {                                     \
-      const unsigned long long t_ = gtimer();                                        \
-      if ((slot) == 0) span_launch_ = atomicAdd(&g_span_entries, 1u) / gridDim.x;    \
-      g_span[blockIdx.x][slot] = t_;                                                 \
-      if ((slot) == 0) {                                                             \
-        unsigned int sm_;                                                            \
-        asm volatile("mov.u32 %0, %%smid;" : "=r"(sm_));                            \
-        g_span_smid[blockIdx.x] = sm_;                                               \
-      }                                                                              \
-      g_span_seq[span_launch_ & 7][blockIdx.x][slot] = t_;                           \
-    }                                                                                \
-  } while (0)
-#define SD_TR(role, j, slot)                                                                        \
-  do {                                                                                              \
-    const int cta_ = blockIdx.x + gridDim.x * blockIdx.y;                                          \
-    if (cta_ < kTraceCtas && (j) < kTraceIters) g_trace[cta_][role][j][slot] = clock64();           \
-  } while (0)
-#else
-constexpr int kTraceLast = 0;
-#define SD_TR(role, j, slot) \
-  do {                       \
-  } while (0)
-#define SD_SPAN(slot) \
-  do {                \
-  } while (0)
-#define SD_SEG(slot) \
-  do {               \
-  } while (0)
-#endif
-#ifdef SD_TRACE
-#define SD_SPAN_DECL __shared__ unsigned int span_launch_
-#else
-#define SD_SPAN_DECL
-#endif
-
-#ifndef SD_EXP_BF16
-#define SD_EXP_BF16 0  // tuning: exp2 of bf16 pairs on the special-function unit (see the exp loop)
-#endif
-
-#ifndef SD_L2_PREFETCH
-#define SD_L2_PREFETCH 0  // prefetch the first tiles into L2 before waiting for the previous kernel
-#endif
-
 #ifndef SD_P_CHUNKED
 #define SD_P_CHUNKED -1  // tuning override of Cfg::CHUNK_P (-1: the per-config choice)
 #endif
@@ -137,19 +74,12 @@ constexpr int kTraceLast = 0;
 #define SD_PING_SHORT 1  // ping-pong also for the single 96-key tile of short key sequences
 #endif
 
-#ifndef SD_SETMAXNREG
-#define SD_SETMAXNREG 0  // 1: move registers from the helper warpgroup to the softmax ones (measured slower)
-#endif
-
-#ifndef SD_MMA_IDLE_NS
-#define SD_MMA_IDLE_NS 0  // backoff of the MMA issuers' idle poll, in ns (0 = spin)
-#endif
-
 #ifndef SD_STAGES_SMALL
 #define SD_STAGES_SMALL 4  // K/V ring depth for head dims <= 64 (one 16 KB K and V tile per stage)
 #endif
 
 constexpr int BM = 128;                               // query rows per tile = TMEM lanes
+enum : int { kSplitPublish = 1, kSplitMerge = 2, kSplitAbort = 3 };  // split hand-off decisions
 constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at B200 clocks
 
 // P_SEP: P has its own TMEM columns (else it overwrites S, and the next S waits for P V).
@@ -184,9 +114,11 @@ struct Cfg {
   static constexpr int V_OFF = K_OFF + STAGES * K_TILE_BYTES;
   static constexpr int BAR_OFF = V_OFF + STAGES * V_TILE_BYTES;
   // q_full, k_full[S], v_full[S], v_ready[S], kv_empty[S], s_full[NQ], s_free[NQ], p_full[NQ], o_done[NQ],
-  // fin[NQ], the exp tokens tok[2][4] of the two tiles' warps on each SM sub-partition, q_empty
-  static constexpr int NBARS = 2 + 4 * STAGES + 5 * NQ + 8 + 2 + 2;
+  // fin[NQ], the exp tokens tok[2][4] of the two tiles' warps on each SM sub-partition, q_empty[2],
+  // split_dec[2], split_written[2]
+  static constexpr int NBARS = 2 + 4 * STAGES + 5 * NQ + 8 + 2 + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  // misc: TMEM base address, abort flag, the split hand-off decisions of the two piece kinds
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
   // TMEM columns of one query tile: S | P (if separate) | O (NPV columns, l at column DH)
   static constexpr int TM_S = 0;
@@ -203,10 +135,6 @@ struct Cfg {
   static constexpr int SOFT_WARP0 = 4;
   static constexpr int NUM_WARPS = 4 + 4 * NQ;
   static constexpr int THREADS = 32 * NUM_WARPS;
-  // Register split for NQ = 2 (setmaxnreg): the helper warpgroup drops to 40 per thread and the two
-  // softmax warpgroups rise to 232; 128 * 40 + 256 * 232 equals the launch budget of 168 x 384.
-  static constexpr int REG_HELPER = 40, REG_SOFT = 232;
-  static_assert(NQ != 2 || 128 * REG_HELPER + 256 * REG_SOFT <= 168 * 384, "register split exceeds the launch budget");
   // Split-item hand-off slot: raw O (NPV fp32 per row) and (m, l) per row of the NQ tiles.
   static constexpr int SLOT_FLOATS = NQ * BM * (NPV + 2);
   // Column pairs after which a softmax warp passes the ping-pong token (measured: half-way for
@@ -241,10 +169,10 @@ struct Bars {
   __device__ uint32_t fin() const { return base + 8 * (2 + 4 * stages + 4 * nq); }
   __device__ uint32_t tok(int t, int q) const { return base + 8 * (2 + 4 * stages + 5 * nq + 4 * t + q); }
   __device__ uint32_t q_empty(int b) const { return base + 8 * (2 + 4 * stages + 5 * nq + 8 + b); }
-  // split-item hand-off: the tail piece's slot is written (all softmax threads), the head piece's
-  // slot may be read (the leader has seen the other CTA's flag)
-  __device__ uint32_t slot_written() const { return base + 8 * (2 + 4 * stages + 5 * nq + 10); }
-  __device__ uint32_t slot_ready() const { return base + 8 * (2 + 4 * stages + 5 * nq + 11); }
+  // split-item hand-off of the tail piece (kind 0) and the head piece (kind 1): the leader's
+  // decision is published, and this piece's slot has been written by every softmax thread
+  __device__ uint32_t split_dec(int kind) const { return base + 8 * (2 + 4 * stages + 5 * nq + 10 + kind); }
+  __device__ uint32_t split_written(int kind) const { return base + 8 * (2 + 4 * stages + 5 * nq + 12 + kind); }
 };
 
 // Bounded wait. Returns false if this CTA has aborted or the limit expired (then it raises the
@@ -286,12 +214,6 @@ struct Part {
 // tensors [B*heads, L, dh] (3-D map); lay_heads = heads: tensors [B, L, heads, dh] (4-D map over
 // {dh, heads, L, B}). Both put the same rows x 128 bytes into shared memory.
 template <bool BLHD>
-__device__ __forceinline__ void prefetch_rows(const CUtensorMap* map, int x, int row, int bh, int lay_heads) {
-  if constexpr (BLHD) tma_prefetch_4d(map, x, bh % lay_heads, row, bh / lay_heads);
-  else tma_prefetch_3d(map, x, row, bh);
-}
-
-template <bool BLHD>
 __device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int row, int bh,
                                           int lay_heads) {
   if constexpr (BLHD) tma_load_4d(dst, map, bar, x, bh % lay_heads, row, bh / lay_heads);
@@ -326,9 +248,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const int nkv = (Lk + BN - 1) / BN;
   const long long u0 = part.u[blockIdx.x], u1 = part.u[blockIdx.x + 1];
 
-  if (threadIdx.x == 0) SD_TR(0, kTraceLast, 0);  // kernel entry (tuning builds only)
-  SD_SPAN_DECL;
-  SD_SPAN(0);
   if (threadIdx.x == 0) {
     mbar_init(bars.q_full(0), 1);
     mbar_init(bars.q_full(1), 1);
@@ -348,8 +267,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     for (int i = 0; i < 8; ++i) mbar_init(bars.tok(i >> 2, i & 3), 1);
     mbar_init(bars.q_empty(0), NQ);
     mbar_init(bars.q_empty(1), NQ);
-    mbar_init(bars.slot_written(), NQ * BM);
-    mbar_init(bars.slot_ready(), 1);
+    for (int kind = 0; kind < 2; ++kind) {
+      mbar_init(bars.split_dec(kind), 1);
+      mbar_init(bars.split_written(kind), NQ * BM);
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -367,28 +288,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // Everything above touched only shared memory, tensor memory and the kernel parameters: it may
-  // overlap the end of the previous kernel on the stream. Global memory waits for that kernel; an
-  // L2 prefetch of this CTA's first Q tiles and K/V tiles is only a hint (it returns no data, and
-  // the loads after the wait read whatever the previous kernel wrote), so it goes first.
-  if (SD_L2_PREFETCH && threadIdx.x == 0 && u0 < u1) {
-    const int it = static_cast<int>(u0 / nkv), kb = static_cast<int>(u0 % nkv);
-    const int bh = it / qpairs, q0 = (it % qpairs) * (BM * NQ);
-    for (int t = 0; t < NQ; ++t)
-      for (int c = 0; c < NCH; ++c) prefetch_rows<C::BLHD>(&tm_q, c * 64, q0 + t * BM, bh, lay_heads);
-    const int ke = static_cast<int>(kb + STAGES < nkv ? kb + STAGES : nkv);
-    for (int j = kb; j < ke && j < kb + (u1 - u0); ++j) {
-      for (int c = 0; c < NCH; ++c) prefetch_rows<C::BLHD>(&tm_k, c * 64, j * BN, bh, lay_heads);
-      for (int c = 0; c < NCHV; ++c) prefetch_rows<C::BLHD>(&tm_v, c * 64, j * BN, bh, lay_heads);
-    }
-  }
+  // overlap the end of the previous kernel on the stream. Global memory waits for that kernel.
   sd::grid_dep_wait();
   sd::grid_dep_launch();
-  if (threadIdx.x == 0) SD_SEG(0);
-  if (threadIdx.x == 0) SD_TR(0, kTraceLast, 1);  // prologue done
 
   if (warp < C::SOFT_WARP0) {
   // ==================================================================== helper warpgroup
-  if (SD_SETMAXNREG && NQ == 2) regs_dec<C::REG_HELPER>();  // registers move to the softmax warpgroups
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -495,7 +400,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           issue_pv(gp % STAGES, jp == 0);
           mma_commit(bars.o_done(t));
           mma_commit(bars.kv_empty(gp % STAGES));
-          SD_TR(warp, gp, 1);
           ++gp;
           if (++jp == sp.ke - sp.kb) {
             have_p = next_seg(up, u1, nkv, sp);
@@ -513,7 +417,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tq = sbase + C::Q_OFF + (qb * NQ + t) * C::Q_TILE_BYTES;
           issue_qk(gq % STAGES);
           mma_commit(bars.s_full(t));
-          SD_TR(warp, gq, 0);
           ++gq;
           if (++jq == sq.ke - sq.kb) {
             mma_commit(bars.q_empty(qb));  // this tile is done reading the segment's Q
@@ -524,7 +427,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           t_idle = clock64();
           continue;
         }
-        if (SD_MMA_IDLE_NS > 0) __nanosleep(SD_MMA_IDLE_NS);  // idle poll: leave issue slots to the softmax
         if ((++spins & 31u) == 0) {
           if (*abort_flag) ok = false;
           else if (clock64() - t_idle > kWaitLimitCycles) {
@@ -561,14 +463,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   }
   tc_fence_before();
   __syncthreads();
-  SD_SPAN(1);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);
   }
   } else {
   // ==================================================================== softmax warpgroups
-  if (SD_SETMAXNREG && NQ == 2) regs_inc<C::REG_SOFT>();
   {
     // ------------------------------------------------------------------ softmax warps
     const int t = (warp - C::SOFT_WARP0) >> 2;  // query tile of this warpgroup
@@ -577,8 +477,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const uint32_t tbase = tmem + t * C::TM_TILE + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t tS = tbase + C::TM_S, tP = tbase + C::TM_P, tO = tbase + C::TM_O;
     bool ok = true;
-    const bool tr = lane == 0;
-    const int trole = warp;
     constexpr bool kPing = SD_PINGPONG && NQ == 2 && (SD_PING_SHORT || BN == 128);
     long long u = u0;
     Seg sg;
@@ -589,13 +487,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     float m_run = -INFINITY, l_run = 0.f;
     for (int j = sg.kb; j < sg.ke; ++j, ++gi) {
       const bool first = j == sg.kb;  // O and l are (re)initialised by this segment's first P V
-      if (tr) SD_TR(trole, gi, 0);
       // warp-uniform outcome: the tcgen05 copies below are .sync.aligned
       if (!__all_sync(0xffffffffu, wait_bar(bars.s_full(t), gi & 1, abort_flag, err))) {
         ok = false;
         break;
       }
-      if (tr) SD_TR(trole, gi, 1);
       tc_fence_after();
       float sv[BN];
 #pragma unroll
@@ -606,7 +502,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(r[i]);
       }
       tmem_wait_ld();
-      if (tr) SD_TR(trole, gi, 2);
       if constexpr (C::P_SEP) {  // S is in registers: the next S = Q K^T may overwrite it
         tc_fence_before();
         mbar_arrive(bars.s_free(t));
@@ -635,7 +530,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // Lazy rescale (always on the first tile). The decision is warp-uniform: the tcgen05 copies
       // of O and l below are .sync.aligned, and rescaling a row whose max barely moved is exact.
       const bool rescale = __any_sync(0xffffffffu, m_new > m_run + 8.0f);
-      if (tr) SD_TR(trole, gi, 3);
       const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
       if (rescale) m_run = m_new;
       // With CHUNK_P, P goes to tensor memory in 16-column chunks as the exp2 loop produces it,
@@ -683,9 +577,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // overlaps the rest of this one (two warps keep the special-function unit busier than one).
       constexpr int kRel = SD_PING_RELEASE >= 0 ? SD_PING_RELEASE : C::PING_RELEASE;
       constexpr int kRelease = kRel > BN / 2 ? BN / 2 : kRel / EB * EB;
-      // Tuning switch: the special-function-unit exponentials on bf16 pairs (argument rounded to
-      // bf16 first). Only where the row sum comes out of P V, which then sums the same bf16 P.
-      constexpr bool kExpBf16 = SD_EXP_BF16 && C::L_IN_V && !C::F16;
 #pragma unroll
       for (int b = 0; b < BN / 2; b += EB) {
         if (kPing && kRelease < BN / 2 && b == kRelease) {
@@ -700,19 +591,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int i = 0; i < EB; ++i) {
           if (((b + i) & 7) < C::POLY_PAIRS) {
             exp2_poly2(x[2 * i], x[2 * i + 1], x[2 * i], x[2 * i + 1]);
-          } else if (!kExpBf16) {
+          } else {
             x[2 * i] = ex2_approx(x[2 * i]);
             x[2 * i + 1] = ex2_approx(x[2 * i + 1]);
           }
         }
 #pragma unroll
         for (int i = 0; i < EB; ++i) {
-          if (kExpBf16 && ((b + i) & 7) >= C::POLY_PAIRS) {
-            pk[b + i] = ex2_bf16x2(pack_bf16x2(x[2 * i], x[2 * i + 1]));
-          } else {
-            if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x[2 * i], x[2 * i + 1]);
-            pk[b + i] = C::F16 ? pack_f16x2(x[2 * i], x[2 * i + 1]) : pack_bf16x2(x[2 * i], x[2 * i + 1]);
-          }
+          if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x[2 * i], x[2 * i + 1]);
+          pk[b + i] = C::F16 ? pack_f16x2(x[2 * i], x[2 * i + 1]) : pack_bf16x2(x[2 * i], x[2 * i + 1]);
         }
         if (kChunkP && (b + EB) % 16 == 0) {  // 16 packed columns done: store them now
           const int c = (b + EB) / 16 - 1;
@@ -727,7 +614,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
       }
-      if (tr) SD_TR(trole, gi, 4);
       // The previous P V (and the O it accumulates) must be complete before P and O are touched.
       if (!kChunkP && C::P_SEP && gi > 0) {
         if (!__all_sync(0xffffffffu, wait_bar(bars.o_done(t), (gi - 1) & 1, abort_flag, err))) {
@@ -736,7 +622,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
         tc_fence_after();
       }
-      if (tr) SD_TR(trole, gi, 5);
       if (!kChunkP && rescale && !first) {
 #pragma unroll
         for (int c = 0; c < C::NPV / 16; ++c) {  // O columns, the row-sum column DH among them
@@ -760,9 +645,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bars.p_full(t));
-      if (tr) SD_TR(trole, gi, 6);
     }
-    if (tr && warp == C::SOFT_WARP0 && sg.ke < nkv && sg.kb == 0) SD_SEG(5);
     if (!ok || !__all_sync(0xffffffffu, wait_bar(bars.o_done(t), (gi - 1) & 1, abort_flag, err))) {
       ok = false;
       break;
@@ -780,79 +663,95 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     float lsum = C::L_IN_V ? ov[C::DH] : l_run;
     const int slot_row = t * BM + row;
-    if (sg.kb > 0) {
-      // Tail piece of an item split with the previous CTA: hand raw O, m and l to it.
-      float* slot = ws + static_cast<size_t>(blockIdx.x - 1) * C::SLOT_FLOATS;
-      float4* dst = reinterpret_cast<float4*>(slot + static_cast<size_t>(slot_row) * C::NPV);
-#pragma unroll
-      for (int i = 0; i < C::NPV / 4; ++i) dst[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
-      float2* ml = reinterpret_cast<float2*>(slot + NQ * BM * C::NPV) + slot_row;
-      *ml = make_float2(m_run, lsum);
-      // Publish: every softmax thread arrives on slot_written (release, CTA scope); one leader
-      // thread -- in the last softmax warp, usually the last to get here -- waits for all of them,
-      // then makes the slot visible device-wide with one fence and one flag increment.
-      mbar_arrive(bars.slot_written());
-      if (warp == C::SOFT_WARP0 + 4 * NQ - 1) {
-        if (!__all_sync(0xffffffffu, wait_bar(bars.slot_written(), 0, abort_flag, err))) {
-          ok = false;
-          break;
+    if (sg.kb > 0 || sg.ke < nkv) {
+      // Split item: a head piece (keys [0, k), at the end of CTA c's range) and a tail piece (keys
+      // [k, nkv), at the start of CTA c+1's range) share one slot and one counter of boundary c.
+      // Whichever piece finishes first claims the slot (counter 0 -> 1), writes its raw O, m and
+      // l there and marks it complete (-> 2); the other piece merges the two and stores O, then
+      // resets the counter for the next launch. No CTA ever waits for another CTA to start: the
+      // only cross-CTA wait is the second finisher's wait for a claimed slot to be completed, by a
+      // CTA that is already running and whose write depends on nothing else.
+      const int kind = sg.ke < nkv ? 1 : 0;  // 1: head piece, 0: tail piece
+      const int bnd = kind ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) - 1;
+      float* slot = ws + static_cast<size_t>(bnd) * C::SLOT_FLOATS;
+      unsigned int* cnt = flags + bnd;
+      volatile int* dec = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 8) + kind;
+      const bool leader_warp = warp == C::SOFT_WARP0 + 4 * NQ - 1;  // usually the last to get here
+      if (leader_warp && lane == 0) {
+        if ((debug_flags & 2) && kind == 0) {  // test hook: hold tail pieces back ~50 us (head finishes first)
+          const long long t0 = clock64();
+          while (clock64() - t0 < 100000) __nanosleep(500);
         }
-        if (lane == 0) {
-          __threadfence();
-          atomicAdd(flags + blockIdx.x - 1, 1u);
-        }
-        __syncwarp();
-      }
-      if (tr && warp == C::SOFT_WARP0) SD_SEG(1 + nseg_done);
-      ++nseg_done;
-      continue;
-    }
-    if (sg.ke < nkv) {
-      // Head piece: wait for the tail (the next CTA processed it at the start of its range), merge.
-      // One leader thread polls the flag, fences, resets the flag for the next launch and opens
-      // slot_ready (acquire/release at CTA scope) for the other softmax threads.
-      float* slot = ws + static_cast<size_t>(blockIdx.x) * C::SLOT_FLOATS;
-      if (tr && warp == C::SOFT_WARP0) SD_SEG(6);
-      if (warp == C::SOFT_WARP0 && lane == 0) {
-        volatile unsigned int* f = flags + blockIdx.x;
-        const long long w0 = clock64();
-        bool got = true;
-        for (uint32_t it = 0; *f == 0u; ++it) {
-          __nanosleep(64);
-          if ((it & 63u) == 63u && (*abort_flag || clock64() - w0 > kWaitLimitCycles)) {
-            if (!*abort_flag) {
-              *abort_flag = 1;
-              atomicOr(err, sd::kDevErrTimeout);
+        int d = kSplitMerge;
+        if (atomicCAS(cnt, 0u, 1u) == 0u) {
+          d = kSplitPublish;
+        } else {  // the other piece claimed the slot: wait until it has been completed
+          volatile unsigned int* f = cnt;
+          const long long w0 = clock64();
+          for (uint32_t it = 0; *f != 2u; ++it) {
+            __nanosleep(32);
+            if ((it & 63u) == 63u && (*abort_flag || clock64() - w0 > kWaitLimitCycles)) {
+              if (!*abort_flag) {
+                *abort_flag = 1;
+                atomicOr(err, sd::kDevErrTimeout);
+              }
+              d = kSplitAbort;
+              break;
             }
-            got = false;
-            break;
           }
-        }
-        if (got) {
           __threadfence();
-          *f = 0u;
-          mbar_arrive(bars.slot_ready());
         }
+        *dec = d;
+        mbar_arrive(bars.split_dec(kind));
       }
       __syncwarp();
-      if (!__all_sync(0xffffffffu, wait_bar(bars.slot_ready(), 0, abort_flag, err))) {
+      if (!__all_sync(0xffffffffu, wait_bar(bars.split_dec(kind), 0, abort_flag, err)) || *dec == kSplitAbort) {
         ok = false;
         break;
       }
-      if (tr && warp == C::SOFT_WARP0) SD_SEG(7);
+      if (*dec == kSplitPublish) {
+        float4* dst = reinterpret_cast<float4*>(slot + static_cast<size_t>(slot_row) * C::NPV);
+#pragma unroll
+        for (int i = 0; i < C::NPV / 4; ++i)
+          dst[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
+        reinterpret_cast<float2*>(slot + NQ * BM * C::NPV)[slot_row] = make_float2(m_run, lsum);
+        // Every softmax thread arrives (release, CTA scope); the leader waits for all of them, then
+        // makes the slot visible device-wide with one fence and marks it complete.
+        mbar_arrive(bars.split_written(kind));
+        if (leader_warp) {
+          if (!__all_sync(0xffffffffu, wait_bar(bars.split_written(kind), 0, abort_flag, err))) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            __threadfence();
+            atomicExch(cnt, 2u);
+          }
+          __syncwarp();
+        }
+        ++nseg_done;
+        continue;
+      }
+      if (leader_warp && lane == 0) atomicExch(cnt, 0u);  // both pieces are done with the counter
+      // Merge in one fixed order, O = O_head * 2^(m_head - m) + O_tail * 2^(m_tail - m), so the result
+      // is the same bit for bit whichever piece merges. The slot is read through L2 only.
       const float4* src = reinterpret_cast<const float4*>(slot + static_cast<size_t>(slot_row) * C::NPV);
-      const float2 ml = reinterpret_cast<const float2*>(slot + NQ * BM * C::NPV)[slot_row];
-      const float m_all = fmaxf(m_run, ml.x);
-      const float a_h = ex2_approx(m_run - m_all), a_t = ex2_approx(ml.x - m_all);
+      const float2 ml = __ldcg(reinterpret_cast<const float2*>(slot + NQ * BM * C::NPV) + slot_row);
+      const float m_head = kind ? m_run : ml.x, m_tail = kind ? ml.x : m_run;
+      const float m_all = fmaxf(m_head, m_tail);
+      const float a_h = ex2_approx(m_head - m_all), a_t = ex2_approx(m_tail - m_all);
+      auto comb = [&](float mine, float theirs) {
+        return kind ? fmaf(mine, a_h, theirs * a_t) : fmaf(theirs, a_h, mine * a_t);
+      };
 #pragma unroll
       for (int i = 0; i < C::NPV / 4; ++i) {
-        const float4 o4 = src[i];
-        ov[4 * i] = ov[4 * i] * a_h + o4.x * a_t;
-        ov[4 * i + 1] = ov[4 * i + 1] * a_h + o4.y * a_t;
-        ov[4 * i + 2] = ov[4 * i + 2] * a_h + o4.z * a_t;
-        ov[4 * i + 3] = ov[4 * i + 3] * a_h + o4.w * a_t;
+        const float4 o4 = __ldcg(src + i);
+        ov[4 * i] = comb(ov[4 * i], o4.x);
+        ov[4 * i + 1] = comb(ov[4 * i + 1], o4.y);
+        ov[4 * i + 2] = comb(ov[4 * i + 2], o4.z);
+        ov[4 * i + 3] = comb(ov[4 * i + 3], o4.w);
       }
-      lsum = C::L_IN_V ? ov[C::DH] : lsum * a_h + ml.y * a_t;
+      lsum = C::L_IN_V ? ov[C::DH] : comb(lsum, ml.y);
     }
     const int qrow = q0 + t * BM + row;
     const float inv_l = 1.0f / lsum;
@@ -870,8 +769,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int i = 0; i < DHP / 8; ++i)
         if (i < n16) dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
     }
-    if (tr) SD_TR(trole, gi - 1, 7);  // segment epilogue done
-    if (tr && warp == C::SOFT_WARP0) SD_SEG(1 + nseg_done);
     ++nseg_done;
     }
   }
@@ -925,10 +822,10 @@ sd_status make_map(CUtensorMap* map, const void* ptr, int64_t dh, int64_t rows, 
 
 int g_debug_flags = 0;
 
-// Per-device hand-off workspace of the persistent schedule (slots of split items + their flags).
-// Allocated on first need and grown, never shrunk; flags start at zero and every launch leaves them
-// at zero. Launches of sd_attention that run concurrently on one device (different streams) must not
-// both split items: they would share the slots.
+// Per-device hand-off workspace of the persistent schedule (slots of split items + their counters).
+// Allocated on first need and grown, never shrunk; counters start at zero and every launch leaves
+// them at zero. Launches of sd_attention that run concurrently on one device (different streams)
+// must not both split items: they would share the slots.
 struct Workspace {
   void* ptr = nullptr;
   size_t bytes = 0;
@@ -982,28 +879,38 @@ namespace {
 
 // Fixed scratch of sd_attention_noalloc: a file-scope device array, so that entry point never
 // allocates. Every device that loads the library holds it until the process exits. Zero at module
-// load; each call clears the hand-off flags it uses before its launch.
+// load; each call clears the hand-off counters it uses before its launch.
 constexpr size_t kFixedScratchBytes = size_t(16) << 20;
 __device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchBytes];
-void* g_fixed_addr[64] = {};
+struct FixedAddr {
+  void* ctx = nullptr;  // the context the address belongs to
+  void* addr = nullptr;
+};
+FixedAddr g_fixed_addr[64];
 std::mutex g_fixed_mu;
 
 // Device address of g_fixed_scratch on the current device. The name of the array in host code is a
-// host-side stand-in, not a device address, so it is resolved once per device with that device
-// current and cached.
+// host-side stand-in, not a device address, so it is resolved with that device current and cached
+// per device, together with the context it was resolved in: if the device's primary context was
+// destroyed and created again (cudaDeviceReset), the address is looked up again.
 sd_status fixed_scratch(void** out) {
   int dev = 0;
   sd_status st = sd::cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
   if (st != SD_OK) return st;
   if (dev >= 64) return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention_noalloc: device index >= 64");
+  void* ctx = nullptr;
+  st = sd::current_context(&ctx);
+  if (st != SD_OK) return st;
   std::lock_guard<std::mutex> lock(g_fixed_mu);
-  if (!g_fixed_addr[dev]) {
+  FixedAddr& f = g_fixed_addr[dev];
+  if (!f.addr || f.ctx != ctx) {
     void* p = nullptr;
     st = sd::cuda_check(cudaGetSymbolAddress(&p, g_fixed_scratch), "cudaGetSymbolAddress(fixed scratch)");
     if (st != SD_OK) return st;
-    g_fixed_addr[dev] = p;
+    f.addr = p;
+    f.ctx = ctx;
   }
-  *out = g_fixed_addr[dev];
+  *out = f.addr;
   return SD_OK;
 }
 
@@ -1107,7 +1014,9 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
     smem_set.fetch_or(bit, std::memory_order_acq_rel);
   }
   // Persistent grid: one CTA per SM (shared memory admits one), each owning an equal share of the
-  // items x K/V-tiles units; items split between two CTAs hand over through the workspace.
+  // items x K/V-tiles units; items split between two CTAs hand over through the workspace. The
+  // hand-off never waits for a CTA to start, so the grid needs no co-residency: CTAs that cannot be
+  // resident at once (SMs held by other work) only run later.
   const int64_t qpairs = (Lq + BM * C::NQ - 1) / (BM * C::NQ);
   const int64_t items = BH * qpairs;
   const int64_t nkv = (Lk + C::BN - 1) / C::BN;
@@ -1137,6 +1046,9 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
   }
   Part part;
   part_ranges(items * nkv, nkv, static_cast<int>(G), CostModel{C::COST_SEG, C::COST_TAIL, C::COST_HEAD}, part.u);
+  for (int64_t c = 0; c < G; ++c)  // the hand-off takes at most two pieces per item
+    if (inside_one_item(part.u[c], part.u[c + 1], nkv))
+      return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention: internal error: a CTA range inside one item");
   const float scale_log2 = scale * 1.4426950408889634f;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(G));
@@ -1228,10 +1140,14 @@ extern "C" sd_status sd_attention_layout(const void* q, const void* k, const voi
 }
 
 // Same computation for callers that cannot allocate device memory (see sd_kernels.h): scratch comes
-// from the fixed file-scope array; the first call on a device resolves its address.
+// from the fixed file-scope array, whose device address every call resolves first (cached per
+// device and context).
 extern "C" sd_status sd_attention_noalloc(const void* q, const void* k, const void* v, void* o, int64_t B,
                                           int64_t heads, int64_t Lq, int64_t Lk, int64_t dh, float scale,
                                           void* stream) {
+  void* p = nullptr;  // resolve the array's address on every call (cached), whatever the shape
+  const sd_status st = fixed_scratch(&p);
+  if (st != SD_OK) return st;
   return attention_impl(q, k, v, o, B, heads, Lq, Lk, dh, scale, stream, true);
 }
 
@@ -1248,31 +1164,6 @@ extern "C" sd_status sd_debug_attention_ranges(int64_t items, int64_t nkv, int64
 }
 
 // Test hook (declared in sd_kernels.h): bit 0 makes the next attention launches skip their first
-// V tile so that the kernel's bounded wait expires and reports SD_ERR_TIMEOUT.
+// V tile so that the kernel's bounded wait expires and reports SD_ERR_TIMEOUT; bit 1 holds the tail
+// pieces of split items back, so that head pieces finish first and the tail pieces merge.
 extern "C" void sd_debug_set_fault(int flags) { g_debug_flags = flags; }
-
-#ifdef SD_TRACE
-// Tuning builds only: copies the phase timestamps to host memory.
-extern "C" int sd_debug_trace(void* host, int64_t bytes) {
-  if (bytes < static_cast<int64_t>(sizeof(g_trace))) return -1;
-  return cudaMemcpyFromSymbol(host, g_trace, sizeof(g_trace)) == cudaSuccess ? 0 : -2;
-}
-extern "C" int sd_debug_span(void* host, int64_t bytes) {
-  if (bytes < static_cast<int64_t>(sizeof(g_span))) return -1;
-  return cudaMemcpyFromSymbol(host, g_span, sizeof(g_span)) == cudaSuccess ? 0 : -2;
-}
-extern "C" int sd_debug_seg(void* host, int64_t bytes) {
-  if (bytes < static_cast<int64_t>(sizeof(g_seg))) return -1;
-  return cudaMemcpyFromSymbol(host, g_seg, sizeof(g_seg)) == cudaSuccess ? 0 : -2;
-}
-extern "C" int sd_debug_span_smid(void* host, int64_t bytes) {
-  if (bytes < static_cast<int64_t>(sizeof(g_span_smid))) return -1;
-  return cudaMemcpyFromSymbol(host, g_span_smid, sizeof(g_span_smid)) == cudaSuccess ? 0 : -2;
-}
-extern "C" int sd_debug_span_seq(void* host, int64_t bytes) {  // and resets the launch counter
-  if (bytes < static_cast<int64_t>(sizeof(g_span_seq))) return -1;
-  if (cudaMemcpyFromSymbol(host, g_span_seq, sizeof(g_span_seq)) != cudaSuccess) return -2;
-  const unsigned int zero = 0;
-  return cudaMemcpyToSymbol(g_span_entries, &zero, sizeof(zero)) == cudaSuccess ? 0 : -3;
-}
-#endif

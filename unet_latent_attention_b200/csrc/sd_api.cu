@@ -14,6 +14,7 @@ __device__ unsigned int g_status_word = 0;
 
 constexpr int kMaxDevices = 64;
 unsigned int* g_status_addr[kMaxDevices] = {};
+void* g_status_ctx[kMaxDevices] = {};  // the context each cached address was resolved in
 int g_sm_count[kMaxDevices] = {};
 std::mutex g_mu;
 
@@ -34,15 +35,36 @@ sd_status cuda_check(cudaError_t err, const char* where) {
   return fail(SD_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(err), cudaGetErrorString(err));
 }
 
+sd_status current_context(void** ctx) {
+  using GetCurrent = int (*)(void**);  // cuCtxGetCurrent(CUcontext*): CUresult
+  static GetCurrent fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GetCurrent>(p);
+  });
+  if (!fn) return fail(SD_ERR_CUDA, "cuCtxGetCurrent is unavailable");
+  *ctx = nullptr;
+  if (fn(ctx) != 0) return fail(SD_ERR_CUDA, "cuCtxGetCurrent failed");
+  return SD_OK;
+}
+
 unsigned int* device_status_word() {
   int dev = 0;
   if (cuda_check(cudaGetDevice(&dev), "cudaGetDevice") != SD_OK || dev >= kMaxDevices) return nullptr;
+  // cudaGetDevice makes the primary context current if none is; the address belongs to it.
+  void* ctx = nullptr;
+  if (current_context(&ctx) != SD_OK) return nullptr;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_status_addr[dev]) {
+  if (!g_status_addr[dev] || g_status_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cuda_check(cudaGetSymbolAddress(&p, g_status_word), "cudaGetSymbolAddress(status)") != SD_OK)
       return nullptr;
     g_status_addr[dev] = static_cast<unsigned int*>(p);
+    g_status_ctx[dev] = ctx;
   }
   return g_status_addr[dev];
 }

@@ -29,6 +29,10 @@ inline bool overlaps(const void* a, int64_t na, const void* b, int64_t nb) {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The calling thread's current CUDA context (as an opaque handle), so that per-device caches of
+// device addresses can notice a context that was destroyed and created again.
+sd_status current_context(void** ctx);
+
 // Streaming-multiprocessor count of the current device (cached per device).
 int sm_count();
 
