@@ -41,6 +41,10 @@ ATTN_SOURCES = ["unet_latent_attention_b200/csrc/attention_sm100.cu", "unet_late
 TRAFFIC_FILE = "profiles/attention_self_sd15_512.md"
 
 
+WORKLOAD_STR = ("SD1.5 512x512 top level: B=2 (CFG pair), Lq=4096 (64x64), C=320, 8 heads dh=40, self Lk=4096, "
+                "cross Lk=77, GroupNorm [2,320,64,64] 32 groups, CFG(w=7.5)+DDIM on [1,4,64,64]")
+
+
 def workload():
     w = si.WORKLOADS[WID]
     attn = dict(w.attention)
@@ -102,14 +106,16 @@ def recorded_traffic():
 
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML while the timed region runs."""
+    """Samples the SM clock and the clock-event reasons through NVML every ~2 ms, from a soak of the
+    same work just before the timed region through the end of the timed region."""
 
     REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
                0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
                0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
     def __init__(self, dev):
-        self.samples, self.reasons, self.ok = [], 0, False
+        self.samples, self.ok = [], False  # (time, MHz, reasons)
+        self.t0 = self.t1 = None
         self._stop = threading.Event()
         try:
             import pynvml
@@ -127,11 +133,18 @@ class ClockSampler:
     def _run(self):
         while not self._stop.is_set():
             try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                self.reasons |= self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, r))
             except Exception:
                 pass
-            time.sleep(0.005)
+            time.sleep(0.002)
+
+    def timed_region(self, start: bool):
+        if start:
+            self.t0 = time.perf_counter()
+        else:
+            self.t1 = time.perf_counter()
 
     def __enter__(self):
         if self.ok:
@@ -147,9 +160,19 @@ class ClockSampler:
     def summary(self):
         if not self.ok:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
-        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
-        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
-                "reasons": names, "samples": len(self.samples)}
+        t0 = self.t0 if self.t0 is not None else float("inf")
+        t1 = self.t1 if self.t1 is not None else float("inf")
+        timed = [m for t, m, _ in self.samples if t0 <= t <= t1 + 0.002]
+        reasons = 0
+        for _, _, r in self.samples:
+            reasons |= r
+        names = [n for b, n in self.REASONS.items() if reasons & b and n != "gpu_idle"]
+        mhz = [m for _, m, _ in self.samples]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(mhz), "samples_in_timed_region": len(timed),
+                "sm_mhz_timed_region": statistics.median(timed) if timed else None,
+                "window": "NVML every ~2 ms over a soak of the same CUDA graph (>= 0.3 s) immediately before "
+                          "the timed region and through it"}
 
 
 # ------------------------------------------------------------------------------------------ ours
@@ -248,12 +271,21 @@ def bench_ours(args, rank, world, dev):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev) as clk:
+        t_soak = time.perf_counter()
+        while time.perf_counter() - t_soak < 0.3:  # soak: the same graph, clocks sampled meanwhile
+            graph_a.replay()
+            torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        clk.timed_region(True)
         t0 = time.perf_counter()
         e_start.record()
         graph_a.replay()
         e_end.record()
         torch.cuda.synchronize()
         wall = time.perf_counter() - t0
+        clk.timed_region(False)
     if world > 1:
         torch.distributed.barrier()
     graph_b.replay()
@@ -303,14 +335,15 @@ def bench_ours(args, rank, world, dev):
 
     e2e = bench_e2e(args, sdk, sets[0], g, a_t, a_p, wl.guidance, flops_step, world, dev)
     extra = {} if args.no_extra else bench_extra(sdk, dev, hbm)
+    configs = [] if args.no_extra else bench_configs(sdk, dev, pk)
     out = {
         "metric": "attention TFLOP/s over the UNet hot-path step (GroupNorm + self-attn + cross-attn + CFG/DDIM)",
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "dtypes": {"attention": "bf16 in, fp32 accumulate", "group_norm": "fp32", "cfg_ddim": "fp32"},
-        "data": "synthetic (seeded torch.randn on device, N(0,1); gamma = 1 + 0.1 N, beta = 0.1 N)",
-        "config": {"workload": wl.name + ": B=2 (CFG pair), Lq=4096 (64x64), C=320, 8 heads dh=40, self Lk=4096, "
-                   "cross Lk=77, GroupNorm [2,320,64,64] 32 groups, CFG(w=7.5)+DDIM on [1,4,64,64]",
+        "data": "synthetic (seeded torch.randn on device, N(0,1); gamma = 1 + 0.1 N, beta = 0.1 N; the CPU arm "
+                "draws the same distributions from synth_inputs)",
+        "config": {"workload": WORKLOAD_STR,
                    "B": 2, "heads": 8, "Lq": 4096, "Lk_self": 4096, "Lk_cross": 77, "dh": 40,
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs rotate over {n_sets} sets of {set_bytes / 2**20:.1f} MiB "
@@ -319,6 +352,7 @@ def bench_ours(args, rank, world, dev):
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": 4 * args.steps,
+        "configs": configs,
         "extra": extra,
         "clocks": clk.summary(),
         "host_wall_s_timed_region": wall,
@@ -326,11 +360,12 @@ def bench_ours(args, rank, world, dev):
     return out, sets
 
 
-def _graph_time_us(fn, n, dev):
-    """Average device time of fn() over n launches captured in one CUDA graph (after warm-up)."""
+def _graph_time_us(fn, n, dev, reps=3):
+    """Device time of one fn(i) averaged over n launches captured in one CUDA graph (after warm-up);
+    the median over `reps` replays, and the replays' total seconds."""
     import torch
-    for _ in range(3):
-        fn(0)
+    for i in range(3):
+        fn(i)
     torch.cuda.synchronize()
     st = torch.cuda.Stream(device=dev)
     gr = torch.cuda.CUDAGraph()
@@ -339,113 +374,200 @@ def _graph_time_us(fn, n, dev):
             fn(i)
     gr.replay()
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    gr.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) * 1e3 / n
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        gr.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1) * 1e3)
+    ts.sort()
+    return ts[len(ts) // 2] / n, ts[len(ts) // 2] * 1e-6
+
+
+def _n_rotating(set_bytes: int, cap: int = 256) -> int:
+    """Number of input/output sets whose total exceeds 2.5x L2, so that a timed sequence of
+    launches over them never re-reads a set from L2."""
+    return max(2, min(cap, math.ceil(2.5 * L2_BYTES / set_bytes)))
+
+
+def _rand(shape, dev, dtype):
+    import torch
+    return torch.randn(shape, device=dev, dtype=torch.float32).to(dtype)
+
+
+def time_attention(sdk, shape, dev, tensor_peak_burst, tensor_peak_sust, hbm):
+    """One attention shape: launches over rotating Q/K/V/O sets (more than 2.5x L2 in total)."""
+    import torch
+    bf = torch.bfloat16
+    B, H, Lq, Lk, dh = shape.B, shape.heads, shape.Lq, shape.Lk, shape.dh
+    set_bytes = 2 * (2 * B * H * Lq * dh + 2 * B * H * Lk * dh)
+    nsets = _n_rotating(set_bytes)
+    sets = [(_rand((B, H, Lq, dh), dev, bf), _rand((B, H, Lk, dh), dev, bf), _rand((B, H, Lk, dh), dev, bf))
+            for _ in range(nsets)]
+    outs = [torch.empty_like(q) for q, _, _ in sets]
+    n = max(nsets, 3 if shape.flops > 2e11 else 20)
+    us, region_s = _graph_time_us(lambda i: sdk.sd_attention(*sets[i % nsets], out=outs[i % nsets]), n, dev)
+    sdk.sd_device_status()
+    tf = shape.flops / (us * 1e-6) / 1e12
+    peak = tensor_peak_sust if region_s > 1.0 else tensor_peak_burst
+    rec = {"shape": [B, H, Lq, Lk, dh], "us": us, "TFLOP/s": tf, "GB/s": set_bytes / (us * 1e-6) / 1e9,
+           "frac_tensor": tf / peak, "frac_hbm": set_bytes / (us * 1e-6) / 1e9 / hbm,
+           "peak_tensor": "sustained" if region_s > 1.0 else "burst", "rotating_sets": nsets,
+           "rotating_MB": nsets * set_bytes / 1e6, "launches": n}
+    del sets, outs
+    torch.cuda.empty_cache()
+    return rec
+
+
+def time_group_norm(sdk, B, C, H, W, dev, hbm, silu_bf16=False):
+    import torch
+    n_el = B * C * H * W
+    byts = (6 if silu_bf16 else 8) * n_el
+    nsets = _n_rotating(byts)
+    xs = [_rand((B, C, H, W), dev, torch.float32) for _ in range(nsets)]
+    ys = [torch.empty(B, C, H, W, device=dev, dtype=torch.bfloat16 if silu_bf16 else torch.float32)
+          for _ in range(nsets)]
+    gm, bt = 1 + 0.1 * torch.randn(C, device=dev), 0.1 * torch.randn(C, device=dev)
+    if silu_bf16:
+        fn = lambda i: sdk.sd_group_norm_silu(xs[i % nsets], gm, bt, 32, 1e-5, out=ys[i % nsets])  # noqa: E731
+    else:
+        fn = lambda i: sdk.sd_group_norm(xs[i % nsets], gm, bt, 32, 1e-5, out=ys[i % nsets])  # noqa: E731
+    us, _ = _graph_time_us(fn, max(nsets, 20), dev)
+    sdk.sd_device_status()
+    gbs = byts / (us * 1e-6) / 1e9
+    del xs, ys
+    torch.cuda.empty_cache()
+    return {"shape": [B, C, H, W], "MB": byts / 1e6, "us": us, "GB/s": gbs, "frac_hbm": gbs / hbm,
+            "rotating_sets": nsets, "rotating_MB": nsets * byts / 1e6}
+
+
+def time_cfg_ddim(sdk, n_el, dev, hbm):
+    import torch
+    byts = 16 * n_el
+    nsets = _n_rotating(byts)
+    sets = [tuple(torch.randn(n_el, device=dev) for _ in range(4)) for _ in range(nsets)]
+    us, _ = _graph_time_us(lambda i: sdk.sd_cfg_ddim_step(*sets[i % nsets][:3], 7.5, 0.3, 0.5,
+                                                          out=sets[i % nsets][3]), max(nsets, 20), dev)
+    sdk.sd_device_status()
+    gbs = byts / (us * 1e-6) / 1e9
+    del sets
+    torch.cuda.empty_cache()
+    return {"elements": n_el, "MB": byts / 1e6, "us": us, "GB/s": gbs, "frac_hbm": gbs / hbm,
+            "rotating_sets": nsets, "rotating_MB": nsets * byts / 1e6}
+
+
+def bench_configs(sdk, dev, pk):
+    """Every configuration of the five workloads at 1 GPU: each attention shape (self and cross),
+    each GroupNorm shape and each workload's guided DDIM step, with rotating inputs larger than L2;
+    attention against the bf16 tensor peak (burst, or sustained for regions over 1 s) and
+    cross-attention / GroupNorm / DDIM against HBM bandwidth."""
+    hbm = pk["hbm_gbs"]
+    out = []
+    for wid, w in si.WORKLOADS.items():
+        rec = {"workload": w.name, "attention": {}, "group_norm": {}}
+        for label, shape in w.attention:
+            rec["attention"][label] = time_attention(sdk, shape, dev, pk["bf16_tflops"], pk["bf16_tflops_sustained"],
+                                                     hbm)
+        for label, g in w.group_norm:
+            rec["group_norm"][label] = time_group_norm(sdk, g.B, g.C, g.H, g.W, dev, hbm)
+        rec["cfg_ddim"] = time_cfg_ddim(sdk, int(np.prod(w.latent)), dev, hbm)
+        rec["cfg_ddim"]["shape"] = list(w.latent)
+        out.append(rec)
+    return out
+
+
+def _loop_sets(lat, n_sets, dev):
+    import torch
+    return [(torch.randn(lat, device=dev), [(torch.randn(lat, device=dev), torch.randn(lat, device=dev))
+                                            for _ in range(20)]) for _ in range(n_sets)]
 
 
 def bench_extra(sdk, dev, hbm):
-    """Labelled extras, not the headline: the 20-step guided DDIM loop of the batched-serving
-    workload (one CUDA graph), a size sweep of GroupNorm and CFG+DDIM up to buffers far larger
-    than L2 that shows the asymptotic HBM bandwidth of these small-shape kernels, the same loop with
-    DPM-Solver++(2M), and cross-attention with longer text contexts."""
+    """Labelled extras, not the headline: the 20-step guided sampling loops of the batched-serving
+    workload (DDIM, DPM-Solver++(2M), third order) as CUDA graphs over independent loop sets whose
+    latents and noise predictions exceed 2.5x L2 in total; a size sweep of GroupNorm (+SiLU),
+    CFG+DDIM and CFG+DPM-Solver++ up to buffers far larger than L2 with rotating inputs; and
+    cross-attention with longer text contexts and fp16 attention."""
     import torch
     out = {}
     lat = si.WORKLOADS[5].latent
-    x = torch.randn(lat, device=dev)
-    eps = [(torch.randn(lat, device=dev), torch.randn(lat, device=dev)) for _ in range(20)]
+    n = int(np.prod(lat))
+    loop_bytes = 41 * 4 * n  # x plus 20 (eps_u, eps_c) pairs
+    nl = _n_rotating(loop_bytes, cap=16)
+    loops = _loop_sets(lat, nl, dev)
     sched = sdk.ddim_schedule(20)
 
-    def loop(_):
+    def loop(i):
+        x, eps = loops[i % nl]
         for (t, a_t, a_p), (eu, ec) in zip(sched, eps):
             sdk.sd_cfg_ddim_step(x, eu, ec, 7.5, a_t, a_p, out=x)
-    us = _graph_time_us(loop, 5, dev)
-    n = int(np.prod(lat))
+    us, _ = _graph_time_us(loop, nl, dev)
     out["cfg_ddim_20_steps_serving"] = {"shape": list(lat), "us_per_loop": us, "us_per_step": us / 20,
-                                        "GB/s": 20 * 16 * n / (us * 1e-6) / 1e9}
-    # the same 20-step guided loop with DPM-Solver++(2M) on Karras sigmas (history buffer in place)
-    hist = torch.zeros(lat, device=dev)
+                                        "GB/s": 20 * 16 * n / (us * 1e-6) / 1e9, "rotating_loops": nl}
+    hists = [torch.zeros(lat, device=dev) for _ in range(nl)]
     dsched = sdk.dpmpp_2m_schedule(20)
 
-    def loop2(_):
+    def loop2(i):
+        x, eps = loops[i % nl]
+        hist = hists[i % nl]
         for (a_p, a_t, a_n, order), (eu, ec) in zip(dsched, eps):
             sdk.sd_cfg_dpmpp_2m_step(x, eu, ec, hist, 7.5, a_p, a_t, a_n, order, out=x, d_out=hist)
-    us = _graph_time_us(loop2, 5, dev)
+    us, _ = _graph_time_us(loop2, nl, dev)
     byts = sum(24 if o == 2 else 20 for *_, o in dsched) * n
     out["cfg_dpmpp_2m_20_steps_serving"] = {"shape": list(lat), "us_per_loop": us, "us_per_step": us / 20,
-                                            "GB/s": byts / (us * 1e-6) / 1e9}
-    # third-order multistep run (orders 1, 2, 3, ..., 3, 1), history rotated through three buffers
-    bufs = [torch.zeros(lat, device=dev) for _ in range(3)]
+                                            "GB/s": byts / (us * 1e-6) / 1e9, "rotating_loops": nl}
+    bufs = [[torch.zeros(lat, device=dev) for _ in range(3)] for _ in range(nl)]
     tsched = sdk.dpmpp_3m_schedule(20)
 
-    def loop3(_):
+    def loop3(j):
+        x, eps = loops[j % nl]
+        b3 = bufs[j % nl]
         for i, ((a2, a1, a_t, a_n, order), (eu, ec)) in enumerate(zip(tsched, eps)):
-            d_out, d1, d2 = bufs[i % 3], bufs[(i - 1) % 3], bufs[(i - 2) % 3]
+            d_out, d1, d2 = b3[i % 3], b3[(i - 1) % 3], b3[(i - 2) % 3]
             if order == 3:
                 sdk.sd_cfg_dpmpp_3m_step(x, eu, ec, d1, d2, 7.5, a2, a1, a_t, a_n, out=x, d_out=d_out)
             else:
                 sdk.sd_cfg_dpmpp_2m_step(x, eu, ec, d1, 7.5, a1, a_t, a_n, order, out=x, d_out=d_out)
-    us = _graph_time_us(loop3, 5, dev)
+    us, _ = _graph_time_us(loop3, nl, dev)
     byts = sum({1: 20, 2: 24, 3: 28}[o] for *_, o in tsched) * n
     out["cfg_dpmpp_3m_20_steps_serving"] = {"shape": list(lat), "us_per_loop": us, "us_per_step": us / 20,
-                                            "GB/s": byts / (us * 1e-6) / 1e9}
+                                            "GB/s": byts / (us * 1e-6) / 1e9, "rotating_loops": nl}
+    del loops, hists, bufs
     sweep = []
     for (B, C, H, W) in [(2, 320, 64, 64), (8, 320, 96, 96), (16, 640, 64, 64), (16, 320, 128, 128)]:
-        xs = [torch.randn(B, C, H, W, device=dev) for _ in range(2)]
-        gm, bt = torch.ones(C, device=dev), torch.zeros(C, device=dev)
-        ys = [torch.empty_like(t) for t in xs]
-        us = _graph_time_us(lambda i: sdk.sd_group_norm(xs[i % 2], gm, bt, 32, 1e-5, out=ys[i % 2]), 20, dev)
-        gbs = 8 * B * C * H * W / (us * 1e-6) / 1e9
-        sweep.append({"kernel": "group_norm", "shape": [B, C, H, W], "MB": 8 * B * C * H * W / 1e6, "us": us,
-                      "GB/s": gbs, "frac_hbm": gbs / hbm})
-        del xs, ys
-    for (B, C, H, W) in [(2, 320, 64, 64), (16, 640, 64, 64)]:  # GroupNorm + SiLU with a bf16 output
-        xs = [torch.randn(B, C, H, W, device=dev) for _ in range(2)]
-        gm, bt = torch.ones(C, device=dev), torch.zeros(C, device=dev)
-        ys = [torch.empty(B, C, H, W, device=dev, dtype=torch.bfloat16) for _ in range(2)]
-        us = _graph_time_us(lambda i: sdk.sd_group_norm_silu(xs[i % 2], gm, bt, 32, 1e-5, out=ys[i % 2]), 20, dev)
-        gbs = 6 * B * C * H * W / (us * 1e-6) / 1e9
-        sweep.append({"kernel": "group_norm_silu_bf16", "shape": [B, C, H, W], "MB": 6 * B * C * H * W / 1e6,
-                      "us": us, "GB/s": gbs, "frac_hbm": gbs / hbm})
-        del xs, ys
+        sweep.append(dict(kernel="group_norm", **time_group_norm(sdk, B, C, H, W, dev, hbm)))
+    for (B, C, H, W) in [(2, 320, 64, 64), (16, 640, 64, 64)]:
+        sweep.append(dict(kernel="group_norm_silu_bf16", **time_group_norm(sdk, B, C, H, W, dev, hbm, True)))
     for m in [1 << 24, 1 << 26]:  # DPM-Solver++(2M), order 2: 24 bytes per element
-        a, u, c, d, o, e = (torch.randn(m, device=dev) for _ in range(6))
-        us = _graph_time_us(lambda i: sdk.sd_cfg_dpmpp_2m_step(a, u, c, d, 7.5, 0.2, 0.3, 0.4, 2, out=o, d_out=e), 20,
-                            dev)
+        nsets = _n_rotating(24 * m)
+        sets = [tuple(torch.randn(m, device=dev) for _ in range(6)) for _ in range(nsets)]
+        us, _ = _graph_time_us(lambda i: sdk.sd_cfg_dpmpp_2m_step(*sets[i % nsets][:4], 7.5, 0.2, 0.3, 0.4, 2,
+                                                                  out=sets[i % nsets][4], d_out=sets[i % nsets][5]),
+                               max(nsets, 20), dev)
         gbs = 24 * m / (us * 1e-6) / 1e9
         sweep.append({"kernel": "cfg_dpmpp_2m", "elements": m, "MB": 24 * m / 1e6, "us": us, "GB/s": gbs,
-                      "frac_hbm": gbs / hbm})
-        del a, u, c, d, o, e
-    for n in [1 << 20, 1 << 24, 1 << 26]:
-        a, u, c, o = (torch.randn(n, device=dev) for _ in range(4))
-        us = _graph_time_us(lambda i: sdk.sd_cfg_ddim_step(a, u, c, 7.5, 0.3, 0.5, out=o), 20, dev)
-        gbs = 16 * n / (us * 1e-6) / 1e9
-        sweep.append({"kernel": "cfg_ddim", "elements": n, "MB": 16 * n / 1e6, "us": us, "GB/s": gbs,
-                      "frac_hbm": gbs / hbm})
-        del a, u, c, o
+                      "frac_hbm": gbs / hbm, "rotating_sets": nsets})
+        del sets
+    for m in [1 << 20, 1 << 24, 1 << 26]:
+        sweep.append(dict(kernel="cfg_ddim", **time_cfg_ddim(sdk, m, dev, hbm)))
+    torch.cuda.empty_cache()
     out["bandwidth_sweep"] = sweep
-    # Cross-attention at the SD1.5 512x512 top level with text contexts of 77, 256 and 512 tokens
-    # (24 rotating input sets, 126 MB of Q per pass: more than L2).
     long = []
     for Lk in (77, 256, 512):
-        sets = [(torch.randn(2, 8, 4096, 40, device=dev, dtype=torch.bfloat16),
-                 torch.randn(2, 8, Lk, 40, device=dev, dtype=torch.bfloat16),
-                 torch.randn(2, 8, Lk, 40, device=dev, dtype=torch.bfloat16)) for _ in range(24)]
-        outs = [torch.empty_like(s[0]) for s in sets]
-        us = _graph_time_us(lambda i: sdk.sd_attention(*sets[i % 24], out=outs[i % 24]), 24, dev)
-        long.append({"shape": [2, 8, 4096, Lk, 40], "us": us, "TFLOP/s": 4 * 2 * 8 * 4096 * Lk * 40 / (us * 1e-6) / 1e12})
-        del sets, outs
+        shape = si.AttnShape(2, 8, 4096, Lk, 40)
+        long.append(time_attention(sdk, shape, dev, 1.0, 1.0, hbm))
+        for k in ("frac_tensor", "peak_tensor"):
+            long[-1].pop(k)
     out["cross_attention_text_length"] = long
-    # fp16 tensors (sd_attention_f16) on the SD1.5 512x512 self- and cross-attention shapes
     f16 = []
-    for Lk in (4096, 77):
+    for Lk in (4096, 77):  # fp16 tensors on the SD1.5 512x512 self- and cross-attention shapes
+        nsets = 12
         sets = [tuple(torch.randn(2, 8, L, 40, device=dev, dtype=torch.float16) for L in (4096, Lk, Lk))
-                for _ in range(12)]
+                for _ in range(nsets)]
         outs = [torch.empty_like(s[0]) for s in sets]
-        us = _graph_time_us(lambda i: sdk.sd_attention(*sets[i % 12], out=outs[i % 12]), 12, dev)
+        us, _ = _graph_time_us(lambda i: sdk.sd_attention(*sets[i % nsets], out=outs[i % nsets]), nsets, dev)
         f16.append({"shape": [2, 8, 4096, Lk, 40], "us": us, "TFLOP/s": 4 * 2 * 8 * 4096 * Lk * 40 / (us * 1e-6) / 1e12})
         del sets, outs
     out["attention_fp16"] = f16
@@ -529,21 +651,50 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def cpu_baseline(budget_s: float):
-    """The oracle as it stands, on a row sample calibrated to take about budget_s."""
-    _, s_self, s_cross, _, _ = workload()
-    flops = attention_flops(s_self) + attention_flops(s_cross)
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _calibrated_sample(budget_s: float):
     rows = 4
     ta, tg, frac = oracle_sample(rows)
     while ta + tg < 0.4 * budget_s and rows < 4096:
         rows = min(4096, int(rows * max(2.0, 0.8 * budget_s / max(ta + tg, 1e-3))))
         ta, tg, frac = oracle_sample(rows)
+    return rows, ta, tg, frac
+
+
+def cpu_baseline(budget_s: float):
+    """The oracle as it stands, on a row sample calibrated to take about budget_s, with the BLAS
+    threads it uses by default; then a smaller sample on one thread for the 1-core figure."""
+    _, s_self, s_cross, _, _ = workload()
+    flops = attention_flops(s_self) + attention_flops(s_cross)
+    rows, ta, tg, frac = _calibrated_sample(0.7 * budget_s)
     full_step_s = ta / frac + tg
-    return {"value": flops / full_step_s / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"{rows} query rows per head (of 4096) of self- and cross-attention for all 16 heads "
-                      f"({ta:.2f} s, scaled by the row fraction {frac:.4f}) plus the whole GroupNorm and CFG+DDIM "
-                      f"({tg:.2f} s), fp64 numpy",
-            "seconds": ta + tg, "full_step_s_estimate": full_step_s}
+    out = {"value": flops / full_step_s / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+           "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
+           "sample": f"{rows} query rows per head (of 4096) of self- and cross-attention for all 16 heads "
+                     f"({ta:.2f} s, scaled by the row fraction {frac:.4f}) plus the whole GroupNorm and CFG+DDIM "
+                     f"({tg:.2f} s), fp64 numpy",
+           "seconds": ta + tg, "full_step_s_estimate": full_step_s}
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            r1, ta1, tg1, frac1 = _calibrated_sample(0.3 * budget_s)
+        step1 = ta1 / frac1 + tg1
+        out["one_core"] = {"value": flops / step1 / 1e12, "unit": "TFLOP/s", "cores": 1,
+                           "full_step_s_estimate": step1,
+                           "sample": f"{r1} query rows per head, scaled by the row fraction {frac1:.5f}"}
+    except Exception as e:  # threadpoolctl missing: no 1-core figure
+        out["one_core"] = {"unavailable": str(e)}
+    return out
 
 
 def bench_reference(args):
@@ -570,9 +721,12 @@ def bench_reference(args):
             "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic (synth_inputs: splitmix64 + Box-Muller, N(0,1))",
-            "config": {"workload": si.WORKLOADS[WID].name + ": B=2, Lq=4096, 8 heads dh=40, self Lk=4096, cross "
-                                                            "Lk=77, GroupNorm [2,320,64,64], CFG+DDIM [1,4,64,64]"},
+            "config": {"workload": WORKLOAD_STR, "B": 2, "heads": 8, "Lq": 4096, "Lk_self": 4096, "Lk_cross": 77,
+                       "dh": 40, "parallelism": "replicas x1",
+                       "inputs": "synth_inputs (splitmix64 + Box-Muller, N(0,1)); the GPU arm draws the same "
+                                 "distributions with torch.randn on the device"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "kind": "oracle", "cores": blas_threads(),
+                             "cpu_model": cpu_model(), "host_cpus": os.cpu_count(),
                              "sample": f"per step: {rows} query rows per head of self- and cross-attention "
                                        f"(scaled by the row fraction {frac:.5f}) plus the whole GroupNorm and "
                                        f"CFG+DDIM, fp64 numpy"},

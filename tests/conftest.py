@@ -14,6 +14,24 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
+# Achieved errors of the GPU parity checks; written as JSON lines to the file named by the
+# SD_PARITY_LOG environment variable at the end of the session (nothing is written without it).
+PARITY_RECORDS = []
+
+
+def record_parity(name, **values):
+    PARITY_RECORDS.append(dict(name=name, **{k: float(v) for k, v in values.items()}))
+
+
+def pytest_sessionfinish(session, exitstatus):
+    path = os.environ.get("SD_PARITY_LOG")
+    if path and PARITY_RECORDS:
+        import json
+        with open(path, "w") as f:
+            for r in PARITY_RECORDS:
+                f.write(json.dumps(r) + "\n")
+
+
 @pytest.fixture(scope="session")
 def golden_dir():
     return GOLDEN

@@ -1,9 +1,14 @@
 """GPU parity of sd_attention against the fp64 oracle on seeded inputs.
 
-Gate (bf16 in, fp32 accumulate): max-abs error <= 2e-2 and mean-abs error <= 2e-3 over the
-compared outputs; sizes span several 128x128 tiles with ragged tails; full workload sizes are
-checked on sampled rows that the oracle computes one by one."""
+Gates (bf16 in, fp32 accumulate), both on every comparison:
+  * the stated tolerance: max-abs error <= 2e-2 and mean-abs error <= 2e-3;
+  * an internal bar: mean-abs error <= 1% of the RMS of the oracle's output over the compared
+    values. At Lk = 4096 |O| is about 0.026 and the stated 2e-3 is ~8% of it; dropping one key tile
+    moves O by ~13x the internal bar (tests/test_oracle_attention.py pins that on the CPU).
+Sizes span several 128x128 tiles with ragged tails; full workload sizes are checked on sampled
+rows that the oracle computes one by one. Achieved errors are logged (SD_PARITY_LOG)."""
 import math
+import os
 
 import numpy as np
 import pytest
@@ -12,11 +17,12 @@ import torch
 import oracle
 import synth_inputs as si
 import unet_latent_attention_b200 as sdk
-from conftest import max_abs_mean_abs
+from conftest import max_abs_mean_abs, record_parity
 
 pytestmark = pytest.mark.gpu
 
 MAX_ABS, MEAN_ABS = 2e-2, 2e-3
+INTERNAL_MEAN_FRAC = 0.01  # internal bar: mean-abs error <= 1% of the output's RMS
 
 
 def _run(q, k, v, dev, scale=None):
@@ -25,10 +31,14 @@ def _run(q, k, v, dev, scale=None):
     return o.float().cpu().numpy()
 
 
-def _check(o, ref, max_abs=MAX_ABS, mean_abs=MEAN_ABS):
+def _check(o, ref, max_abs=MAX_ABS, mean_abs=MEAN_ABS, name=None):
     mx, mn = max_abs_mean_abs(o, ref)
+    rms = float(np.sqrt(np.mean(np.square(np.asarray(ref, np.float64))))) if np.size(ref) else 0.0
     assert np.isfinite(o).all()
+    record_parity(name or os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0], max_abs=mx, mean_abs=mn,
+                  rms_ref=rms)
     assert mx <= max_abs and mn <= mean_abs, (mx, mn)
+    assert mn <= INTERNAL_MEAN_FRAC * rms, ("internal bar", mn, rms)
     return mx, mn
 
 

@@ -136,3 +136,28 @@ def test_bf16_inputs_are_taken_exactly():
     o = oracle.attention(q16, k16, v16)
     o2 = oracle.attention(q16.double().numpy(), k16.double().numpy(), v16.double().numpy())
     np.testing.assert_array_equal(o, o2)
+
+
+# ---- the internal parity bar of the GPU tests (mean-abs error <= 1% of the RMS of the output)
+
+INTERNAL_MEAN_FRAC = 0.01
+
+
+@pytest.mark.parametrize("Lk", [4096, 77])
+def test_internal_bar_detects_a_dropped_key_tile(Lk):
+    # The GPU parity tests gate mean-abs error at 1% of the oracle output's RMS, besides the stated
+    # 2e-3. At Lk = 4096 with N(0,1) inputs, |O| is about 0.026, so 2e-3 alone is ~8% of the signal.
+    # A kernel that skipped one 128-key tile (or, at Lk = 77, one 16-key MMA slice) would move O by
+    # far more than the internal bar; this pins that the bar can see such a slip.
+    q = normal((1, 1, 64, 40), 71).astype(np.float32)
+    k = normal((1, 1, Lk, 40), 72).astype(np.float32)
+    v = normal((1, 1, Lk, 40), 73).astype(np.float32)
+    o = oracle.attention(q, k, v)
+    drop = slice(128, 256) if Lk > 128 else slice(16, 32)
+    keep = np.ones(Lk, bool)
+    keep[drop] = False
+    o_drop = oracle.attention(q, k[:, :, keep], v[:, :, keep], scale=1 / math.sqrt(40))
+    bar = INTERNAL_MEAN_FRAC * float(np.sqrt(np.mean(o ** 2)))
+    shift = float(np.abs(o_drop - o).mean())
+    assert shift > 5 * bar, (shift, bar)
+    assert bar < 2e-3  # tighter than the stated gate on these shapes

@@ -153,9 +153,6 @@ __device__ __forceinline__ void cluster_group_stats(Stats st, float eps, float* 
 #ifndef SD_GN_MINB
 #define SD_GN_MINB 1
 #endif
-#ifndef SD_GN_STREAM_BIG
-#define SD_GN_STREAM_BIG 0  // tuning: groups that need 512+ thread CTAs take the streaming path
-#endif
 
 template <int ITEMS, int THREADS, int EPI>
 __global__ void __launch_bounds__(THREADS, (SD_GN_MINB && THREADS == 512 && ITEMS <= 10) ? 2 : 1) gn_resident(const float* x, const float* __restrict__ gamma,
@@ -340,7 +337,6 @@ sd_status group_norm_impl(const char* name, const float* x, const float* gamma, 
     const int* tl = SD_GN_POLICY == 0 ? tlist0 : tlist1;
     for (int ti = 0; ti < 3 && !cs; ++ti) {
       const int th = tl[ti];
-      if (SD_GN_STREAM_BIG && th >= 512) break;
       const int max_items = th == 1024 ? 8 : kMaxItems;
       for (int c = 1; c <= kMaxCluster; c *= 2) {
         if (group_elems % (4 * c) != 0 || group_elems / c > int64_t(th) * 4 * max_items) continue;
