@@ -88,13 +88,16 @@ sd_status sd_group_norm_silu(const float* x, const float* gamma, const float* be
  * Attention, "从零实现扩散模型推理引擎：Rust + wgpu 的 GPU 加速图像生成架构" §3.2: for each batch b, head h
  * and query row i, O[b,h,i,:] = sum_j softmax_j(scale * Q[b,h,i,:] . K[b,h,j,:]) V[b,h,j,:].
  * The kernel is a flash-style forward pass (tiles of 128 queries x 128 keys, running max and
- * running sum, normalisation at the end) on the sm_100a tensor cores with fp32 accumulation.
+ * running sum, normalisation at the end) on the sm_100a tensor cores with fp32 accumulation. For
+ * Lk <= 80 (the 77-token text context) a second kernel keeps all of K and V resident in shared
+ * memory and takes one exact softmax pass per 128-row query tile (§3.2's cross-attention).
  *  q      : bf16 [B, heads, Lq, dh] contiguous.
  *  k, v   : bf16 [B, heads, Lk, dh] contiguous (self-attention: Lk = Lq = H*W;
  *           cross-attention: Lk = 77 text tokens, already projected to heads x dh).
  *  o      : bf16 [B, heads, Lq, dh] contiguous; must not overlap q, k or v.
  *  dh     : one of 40, 64, 80, 160 (SD1.5 and SDXL head sizes); others are SD_ERR_UNSUPPORTED.
- *  scale  : finite; callers normally pass 1/sqrt(dh).
+ *  scale  : finite and >= 0 (SD_ERR_INVALID_ARG if not finite, SD_ERR_UNSUPPORTED if negative);
+ *           callers normally pass 1/sqrt(dh).
  *  Lq, Lk : >= 1 and <= 2^30, any value (ragged tails are masked). B*heads < 2^31.
  * All four pointers must be 16-byte aligned (SD_ERR_MISALIGNED otherwise).
  * Scratch: when a shape has more query-tile items than the GPU has SMs, some items are split

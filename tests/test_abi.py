@@ -38,6 +38,7 @@ def test_attention_argument_errors(L):
     assert L.sd_attention(P, P, P, P, 1, 1, 8, 8, 50, 1.0, None) == 2 and "head dim" in _err(L)
     assert L.sd_attention(P, P, P, P, -1, 1, 8, 8, 40, 1.0, None) == 1
     assert L.sd_attention(P, P, P, P, 1, 1, 8, 8, 40, float("nan"), None) == 1
+    assert L.sd_attention(P, P, P, P, 1, 1, 8, 8, 40, -0.5, None) == 2 and "negative scale" in _err(L)
     assert L.sd_attention(P + 2, P, P, P, 1, 1, 8, 8, 40, 1.0, None) == 3
     assert L.sd_attention(P, P, P, P + 64, 1, 1, 8, 8, 40, 1.0, None) == 1 and "overlap" in _err(L)
     assert L.sd_attention(0, 0, 0, 0, 0, 8, 8, 8, 40, 1.0, None) == 0  # empty: no launch

@@ -41,10 +41,62 @@
 
 #include "sd_internal.h"
 #include "sm100_ptx.cuh"
+#include "attn_common.cuh"
+
+namespace sd {
+namespace attn {
+
+int g_debug_flags = 0;
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+sd_status make_map(CUtensorMap* map, const void* ptr, int64_t dh, int64_t rows, int64_t planes, int box_rows,
+                   bool f16, int64_t lay_heads) {
+  auto fn = encode_fn();
+  if (!fn) return sd::fail(SD_ERR_CUDA, "sd_attention: cuTensorMapEncodeTiled is unavailable");
+  const cuuint32_t rank = lay_heads ? 4 : 3;
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4];
+  if (lay_heads) {
+    dims[0] = dh, dims[1] = lay_heads, dims[2] = rows, dims[3] = planes / lay_heads;
+    strides[0] = dh * 2, strides[1] = lay_heads * dh * 2, strides[2] = rows * lay_heads * dh * 2;
+    box[0] = 64, box[1] = 1, box[2] = static_cast<cuuint32_t>(box_rows), box[3] = 1;
+  } else {
+    dims[0] = dh, dims[1] = rows, dims[2] = planes;
+    strides[0] = dh * 2, strides[1] = rows * dh * 2;
+    box[0] = 64, box[1] = static_cast<cuuint32_t>(box_rows), box[2] = 1;
+  }
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
+                        const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return sd::fail(SD_ERR_CUDA, "sd_attention: cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return SD_OK;
+}
+
+
+}  // namespace attn
+}  // namespace sd
 
 namespace {
 
 using namespace sm100;
+using namespace sd::attn;
+
+enum : int { kSplitPublish = 1, kSplitMerge = 2, kSplitAbort = 3 };  // split hand-off decisions
 
 #ifndef SD_POLY_PAIRS
 #define SD_POLY_PAIRS -1  // tuning override of the per-head-dim choice in the launch table
@@ -78,9 +130,6 @@ using namespace sm100;
 #define SD_STAGES_SMALL 4  // K/V ring depth for head dims <= 64 (one 16 KB K and V tile per stage)
 #endif
 
-constexpr int BM = 128;                               // query rows per tile = TMEM lanes
-enum : int { kSplitPublish = 1, kSplitMerge = 2, kSplitAbort = 3 };  // split hand-off decisions
-constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at B200 clocks
 
 // P_SEP: P has its own TMEM columns (else it overwrites S, and the next S waits for P V).
 // L_IN_V: the softmax row sums come out of the P V product itself: a fix-up warp writes bf16 1.0
@@ -175,25 +224,6 @@ struct Bars {
   __device__ uint32_t split_written(int kind) const { return base + 8 * (2 + 4 * stages + 5 * nq + 12 + kind); }
 };
 
-// Bounded wait. Returns false if this CTA has aborted or the limit expired (then it raises the
-// CTA's abort flag and the device status word). `abortable = false` is for teardown drains.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, unsigned int* err,
-                                      bool abortable = true) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 127u) == 0) {
-      if (abortable && *abort_flag) return false;
-      if (clock64() - t0 > kWaitLimitCycles) {
-        *abort_flag = 1;
-        atomicOr(err, sd::kDevErrTimeout);
-        return false;
-      }
-    }
-  }
-}
-
 // Persistent schedule: the work is items x nkv units (an item = NQ query tiles of one (b, h); a
 // unit = one K/V tile of it). CTA c owns units [c U / G, (c+1) U / G) in item-major order, so every
 // CTA gets the same amount of work whatever the number of SMs; with G <= items each range spans at
@@ -213,12 +243,6 @@ struct Part {
 // One tile of rows [row, row + box) of head plane bh, 64 head-dim columns from x. lay_heads = 0:
 // tensors [B*heads, L, dh] (3-D map); lay_heads = heads: tensors [B, L, heads, dh] (4-D map over
 // {dh, heads, L, B}). Both put the same rows x 128 bytes into shared memory.
-template <bool BLHD>
-__device__ __forceinline__ void load_rows(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int row, int bh,
-                                          int lay_heads) {
-  if constexpr (BLHD) tma_load_4d(dst, map, bar, x, bh % lay_heads, row, bh / lay_heads);
-  else tma_load_3d(dst, map, bar, x, row, bh);
-}
 __device__ __forceinline__ bool next_seg(long long& u, long long u1, int nkv, Seg& sg) {
   if (u >= u1) return false;
   sg.it = static_cast<int>(u / nkv);
@@ -778,49 +802,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// 3-D map over a contiguous bf16 [planes, rows, dh] tensor, box {64, box_rows, 1}, 128-byte swizzle.
-// lay_heads = 0: [planes, rows, dh]; lay_heads = heads: [planes / heads, rows, heads, dh] as the 4-D
-// map {dh, heads, rows, B} with box {64, 1, box_rows, 1}.
-sd_status make_map(CUtensorMap* map, const void* ptr, int64_t dh, int64_t rows, int64_t planes, int box_rows,
-                   bool f16, int64_t lay_heads = 0) {
-  auto fn = encode_fn();
-  if (!fn) return sd::fail(SD_ERR_CUDA, "sd_attention: cuTensorMapEncodeTiled is unavailable");
-  const cuuint32_t rank = lay_heads ? 4 : 3;
-  cuuint64_t dims[4], strides[3];
-  cuuint32_t box[4];
-  if (lay_heads) {
-    dims[0] = dh, dims[1] = lay_heads, dims[2] = rows, dims[3] = planes / lay_heads;
-    strides[0] = dh * 2, strides[1] = lay_heads * dh * 2, strides[2] = rows * lay_heads * dh * 2;
-    box[0] = 64, box[1] = 1, box[2] = static_cast<cuuint32_t>(box_rows), box[3] = 1;
-  } else {
-    dims[0] = dh, dims[1] = rows, dims[2] = planes;
-    strides[0] = dh * 2, strides[1] = rows * dh * 2;
-    box[0] = 64, box[1] = static_cast<cuuint32_t>(box_rows), box[2] = 1;
-  }
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  const CUresult r = fn(map, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
-                        const_cast<void*>(ptr), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return sd::fail(SD_ERR_CUDA, "sd_attention: cuTensorMapEncodeTiled failed (%d)", (int)r);
-  return SD_OK;
-}
-
-int g_debug_flags = 0;
 
 // Per-device hand-off workspace of the persistent schedule (slots of split items + their counters).
 // Allocated on first need and grown, never shrunk; counters start at zero and every launch leaves
@@ -995,9 +976,9 @@ template <class C>
 sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t BH, int64_t Lq, int64_t Lk,
                  int64_t dh, float scale, cudaStream_t s, bool fixed, int64_t lay_heads) {
   CUtensorMap mq, mk, mv;
-  sd_status st = make_map(&mq, q, dh, Lq, BH, BM, C::F16, lay_heads);
-  if (st == SD_OK) st = make_map(&mk, k, dh, Lk, BH, C::BN, C::F16, lay_heads);
-  if (st == SD_OK) st = make_map(&mv, v, dh, Lk, BH, C::BN, C::F16, lay_heads);
+  sd_status st = sd::attn::make_map(&mq, q, dh, Lq, BH, BM, C::F16, lay_heads);
+  if (st == SD_OK) st = sd::attn::make_map(&mk, k, dh, Lk, BH, C::BN, C::F16, lay_heads);
+  if (st == SD_OK) st = sd::attn::make_map(&mv, v, dh, Lk, BH, C::BN, C::F16, lay_heads);
   if (st != SD_OK) return st;
   unsigned int* err = sd::device_status_word();
   if (!err) return SD_ERR_CUDA;
@@ -1060,7 +1041,7 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
   cfg.numAttrs = sd::pdl_attr(&attr[0]);
   return sd::cuda_check(
       cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, static_cast<uint16_t*>(o), static_cast<int>(Lq),
-                         static_cast<int>(Lk), static_cast<int>(dh), scale_log2, err, g_debug_flags,
+                         static_cast<int>(Lk), static_cast<int>(dh), scale_log2, err, sd::attn::g_debug_flags,
                          static_cast<int>(qpairs), static_cast<int>(items), ws, flags, static_cast<int>(lay_heads),
                          part),
       "sd_attention launch");
@@ -1074,7 +1055,9 @@ namespace {
 template <bool F16, bool BLHD>
 sd_status dispatch(const void* q, const void* k, const void* v, void* o, int64_t BH, int64_t Lq, int64_t Lk,
                    int64_t dh, float scale, cudaStream_t s, bool fixed, int64_t lay_heads) {
-  if (Lk <= 96) {  // short key sequence (the 77-token text context): one 96-key tile, no online rescale
+  // Short key sequences (the 77-token text context): all of K and V resident, one exact softmax pass.
+  if (Lk <= sd::attn::kShortMaxKeys) return sd::attn::launch_short(q, k, v, o, BH, Lq, Lk, dh, scale, s, F16, lay_heads);
+  if (Lk <= 96) {  // one 96-key tile, no online rescale
     switch (dh) {
       case 40: return launch<Cfg<40, 96, SD_CROSS_NQ, 2, true, true, 0, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
       case 64: return launch<Cfg<64, 96, SD_CROSS_NQ, 2, true, false, 0, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
@@ -1097,6 +1080,9 @@ sd_status attention_impl(const void* q, const void* k, const void* v, void* o, i
   if (dh != 40 && dh != 64 && dh != 80 && dh != 160)
     return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention: head dim %lld not in {40, 64, 80, 160}", (long long)dh);
   if (!std::isfinite(scale)) return sd::fail(SD_ERR_INVALID_ARG, "sd_attention: scale is not finite");
+  // The kernels take each row's maximum score times the scale as the softmax shift, which is the
+  // maximum of the scaled scores only for scale >= 0.
+  if (scale < 0.f) return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention: negative scale");
   if (B == 0 || heads == 0 || Lq == 0) return SD_OK;
   if (Lk == 0) return sd::fail(SD_ERR_INVALID_ARG, "sd_attention: Lk must be >= 1 when Lq >= 1");
   if (!q || !k || !v || !o) return sd::fail(SD_ERR_INVALID_ARG, "sd_attention: null pointer");
@@ -1166,4 +1152,4 @@ extern "C" sd_status sd_debug_attention_ranges(int64_t items, int64_t nkv, int64
 // Test hook (declared in sd_kernels.h): bit 0 makes the next attention launches skip their first
 // V tile so that the kernel's bounded wait expires and reports SD_ERR_TIMEOUT; bit 1 holds the tail
 // pieces of split items back, so that head pieces finish first and the tail pieces merge.
-extern "C" void sd_debug_set_fault(int flags) { g_debug_flags = flags; }
+extern "C" void sd_debug_set_fault(int flags) { sd::attn::g_debug_flags = flags; }
