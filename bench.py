@@ -733,6 +733,53 @@ def bench_reference(args):
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def profile_case(spec: str, launches: int) -> None:
+    """Runs `launches` launches of one kernel on one shape and nothing else, for ncu captures:
+    attn:B,H,Lq,Lk,dh | gn:B,C,H,W | gn_silu:B,C,H,W | ddim:n | dpmpp2:n (rotating inputs over 2.5x L2)."""
+    import torch
+    import unet_latent_attention_b200 as sdk
+    from unet_latent_attention_b200 import build
+    build.build()
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    kind, dims = spec.split(":")
+    d = [int(x) for x in dims.split(",")]
+    if kind == "attn":
+        B, H, Lq, Lk, dh = d
+        nsets = _n_rotating(2 * (2 * B * H * Lq * dh + 2 * B * H * Lk * dh), cap=8)
+        sets = [(_rand((B, H, Lq, dh), dev, torch.bfloat16), _rand((B, H, Lk, dh), dev, torch.bfloat16),
+                 _rand((B, H, Lk, dh), dev, torch.bfloat16)) for _ in range(nsets)]
+        outs = [torch.empty_like(q) for q, _, _ in sets]
+        fn = lambda i: sdk.sd_attention(*sets[i % nsets], out=outs[i % nsets])  # noqa: E731
+    elif kind in ("gn", "gn_silu"):
+        B, C, H, W = d
+        nsets = _n_rotating(8 * B * C * H * W, cap=8)
+        xs = [_rand((B, C, H, W), dev, torch.float32) for _ in range(nsets)]
+        ys = [torch.empty(B, C, H, W, device=dev, dtype=torch.bfloat16 if kind == "gn_silu" else torch.float32)
+              for _ in range(nsets)]
+        gm, bt = torch.ones(C, device=dev), torch.zeros(C, device=dev)
+        if kind == "gn":
+            fn = lambda i: sdk.sd_group_norm(xs[i % nsets], gm, bt, 32, 1e-5, out=ys[i % nsets])  # noqa: E731
+        else:
+            fn = lambda i: sdk.sd_group_norm_silu(xs[i % nsets], gm, bt, 32, 1e-5, out=ys[i % nsets])  # noqa: E731
+    elif kind in ("ddim", "dpmpp2"):
+        n = d[0]
+        per = 16 if kind == "ddim" else 24
+        nsets = _n_rotating(per * n, cap=8)
+        sets = [tuple(torch.randn(n, device=dev) for _ in range(6)) for _ in range(nsets)]
+        if kind == "ddim":
+            fn = lambda i: sdk.sd_cfg_ddim_step(*sets[i % nsets][:3], 7.5, 0.3, 0.5, out=sets[i % nsets][3])  # noqa: E731
+        else:
+            fn = lambda i: sdk.sd_cfg_dpmpp_2m_step(*sets[i % nsets][:4], 7.5, 0.2, 0.3, 0.4, 2,  # noqa: E731
+                                                    out=sets[i % nsets][4], d_out=sets[i % nsets][5])
+    else:
+        raise SystemExit(f"unknown profile case {spec}")
+    for i in range(launches):
+        fn(i)
+    sdk.sd_device_status()
+    print(f"profiled {spec}: {launches} launches")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -742,7 +789,13 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the labelled DDIM-loop and bandwidth-sweep extras")
+    ap.add_argument("--profile", default="", help="run only `--launches` launches of one kernel (for ncu): "
+                                                   "attn:B,H,Lq,Lk,dh | gn:B,C,H,W | gn_silu:B,C,H,W | ddim:n | dpmpp2:n")
+    ap.add_argument("--launches", type=int, default=3)
     args = ap.parse_args()
+    if args.profile:
+        profile_case(args.profile, args.launches)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 

@@ -151,6 +151,18 @@ def test_repeated_launches_reuse_the_hand_off_flags(cuda):
         _check(o.float().cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("dh", [40, 64, 80, 160])
+@pytest.mark.parametrize("B,heads,Lq,Lk", [(2, 300, 100, 77), (1, 7, 1000, 80), (2, 4, 200, 81), (3, 5, 1, 77),
+                                           (2, 37, 129, 50)])
+def test_short_key_sequences(cuda, dh, B, heads, Lq, Lk):
+    # Lk <= 80 takes the resident-K/V kernel: CTA ranges that cross several heads (K/V buffers
+    # reused), the 80-key boundary, a single query row, ragged query tiles; Lk = 81 takes the
+    # general kernel's 96-key tile
+    q, k, v = _qkv(B, heads, Lq, Lk, dh, 9300 + dh + Lq + Lk)
+    o = _run(q, k, v, cuda)
+    _check(o, oracle.attention(q, k, v))
+
+
 LONG_TEXT = [si.AttnShape(2, 8, 4096, 256, 40), si.AttnShape(2, 8, 4096, 512, 40),
              si.AttnShape(2, 10, 1024, 256, 64), si.AttnShape(2, 10, 1024, 512, 64)]
 

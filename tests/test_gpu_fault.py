@@ -1,5 +1,5 @@
-"""Failure path on the GPU without a fault: the test hook makes one attention launch skip its
-first V tile, so the kernel's bounded mbarrier wait expires (after about a second). The kernel
+"""Failure path on the GPU without a fault: the test hook makes one attention launch (the general
+kernel, and the short-key-sequence kernel) skip its first V tile, so the kernel's bounded mbarrier wait expires (after about a second). The kernel
 must drain its own copies and MMAs, free tensor memory, return, and report SD_ERR_TIMEOUT through
 sd_device_status; the context stays usable and the next launch is correct. Runs in a child
 process with a timeout so that a regression cannot hold the test session."""
@@ -19,8 +19,8 @@ CHILD = textwrap.dedent(r"""
     import unet_latent_attention_b200 as sdk
     dev = torch.device("cuda:0")
     q = si.to_bf16_exact(si.normal((1, 1, 128, 64), 11)).to(dev)
-    k = si.to_bf16_exact(si.normal((1, 1, 256, 64), 12)).to(dev)
-    v = si.to_bf16_exact(si.normal((1, 1, 256, 64), 13)).to(dev)
+    k = si.to_bf16_exact(si.normal((1, 1, {lk}, 64), 12)).to(dev)
+    v = si.to_bf16_exact(si.normal((1, 1, {lk}, 64), 13)).to(dev)
     sdk.sd_device_status()
     sdk.sd_debug_set_fault(1)
     sdk.sd_attention(q, k, v)
@@ -39,8 +39,10 @@ CHILD = textwrap.dedent(r"""
 """)
 
 
-def test_bounded_wait_reports_timeout(cuda):
+@pytest.mark.parametrize("lk", [256, 77], ids=["general-kernel", "short-key-kernel"])
+def test_bounded_wait_reports_timeout(cuda, lk):
     import os
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    r = subprocess.run([sys.executable, "-c", CHILD.format(root=root)], capture_output=True, text=True, timeout=90)
+    r = subprocess.run([sys.executable, "-c", CHILD.format(root=root, lk=lk)], capture_output=True, text=True,
+                       timeout=90)
     assert r.returncode == 0 and "FAULT_PATH_OK" in r.stdout, (r.stdout[-2000:], r.stderr[-2000:])

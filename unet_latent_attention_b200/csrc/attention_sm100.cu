@@ -110,6 +110,10 @@ enum : int { kSplitPublish = 1, kSplitMerge = 2, kSplitAbort = 3 };  // split ha
 #define SD_PING_RELEASE -1  // tuning override of Cfg::PING_RELEASE (-1: the per-config choice)
 #endif
 
+#ifndef SD_EXP_SPLIT
+#define SD_EXP_SPLIT 1  // special-function pairs before the token hand-off, polynomial pairs after
+#endif
+
 #ifndef SD_PINGPONG
 #define SD_PINGPONG 1  // alternate the two query tiles' exp2 phases on each SM sub-partition
 #endif
@@ -601,8 +605,35 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // overlaps the rest of this one (two warps keep the special-function unit busier than one).
       constexpr int kRel = SD_PING_RELEASE >= 0 ? SD_PING_RELEASE : C::PING_RELEASE;
       constexpr int kRelease = kRel > BN / 2 ? BN / 2 : kRel / EB * EB;
+      // Split order: the special-function-unit pairs first, then the token, then the FMA-pipe
+      // polynomial pairs, so that this warp's polynomial work overlaps the partner warp's
+      // special-function phase instead of lengthening the phase that holds the token.
+      constexpr bool kSplit = SD_EXP_SPLIT && kPing && C::POLY_PAIRS > 0 && !kChunkP;
+      if constexpr (kSplit) {
 #pragma unroll
-      for (int b = 0; b < BN / 2; b += EB) {
+        for (int b = 0; b < BN / 2; ++b) {
+          if ((b & 7) < C::POLY_PAIRS) continue;
+          float x0, x1;
+          fma2(x0, x1, sv[2 * b], sv[2 * b + 1], scale_log2, scale_log2, neg_m, neg_m);
+          x0 = ex2_approx(x0);
+          x1 = ex2_approx(x1);
+          if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x0, x1);
+          pk[b] = C::F16 ? pack_f16x2(x0, x1) : pack_bf16x2(x0, x1);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
+#pragma unroll
+        for (int b = 0; b < BN / 2; ++b) {
+          if ((b & 7) >= C::POLY_PAIRS) continue;
+          float x0, x1;
+          fma2(x0, x1, sv[2 * b], sv[2 * b + 1], scale_log2, scale_log2, neg_m, neg_m);
+          exp2_poly2(x0, x1, x0, x1);
+          if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x0, x1);
+          pk[b] = C::F16 ? pack_f16x2(x0, x1) : pack_bf16x2(x0, x1);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < BN / 2 && !kSplit; b += EB) {
         if (kPing && kRelease < BN / 2 && b == kRelease) {
           __syncwarp();
           if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
@@ -634,7 +665,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
       }
       if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
-      if (kPing && kRelease == BN / 2) {
+      if (kPing && kRelease == BN / 2 && !kSplit) {
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
       }
