@@ -30,6 +30,10 @@
 #include "sd_internal.h"
 #include "sm100_ptx.cuh"
 
+#ifndef SD_SHORT_POLY
+#define SD_SHORT_POLY 2
+#endif
+
 namespace {
 
 using namespace sm100;
@@ -41,6 +45,7 @@ struct ShortCfg {
   static constexpr bool F16 = F16_;
   static constexpr bool BLHD = BLHD_;
   static constexpr int BN = kShortMaxKeys;             // keys in the resident tile
+  static constexpr int POLY = SD_SHORT_POLY;           // of every 8 column pairs, exp2 on the FMA pipe
   static constexpr int DHP = (DH + 15) / 16 * 16;      // Q K^T depth padded to the MMA granule
   static constexpr int NPV = (DH + 1 + 15) / 16 * 16;  // N of O = P V: O columns, then the row sum at DH
   static constexpr int NCH = (DHP + 63) / 64;          // 128-byte swizzle chunks of Q and K rows
@@ -343,8 +348,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int b = 0; b < BN / 2; ++b) {
         float x0, x1;
         fma2(x0, x1, sv[2 * b], sv[2 * b + 1], scale_log2, scale_log2, neg_m, neg_m);
-        x0 = ex2_approx(x0);
-        x1 = ex2_approx(x1);
+        if ((b & 7) < C::POLY) {  // FMA-pipe exp2 for POLY of every 8 pairs, the rest on the SFU
+          exp2_poly2(x0, x1, x0, x1);
+        } else {
+          x0 = ex2_approx(x0);
+          x1 = ex2_approx(x1);
+        }
         pk[b] = C::F16 ? pack_f16x2(x0, x1) : pack_bf16x2(x0, x1);
       }
       // P over S: the scores are in registers, so the slot's first BN/2 columns take P
