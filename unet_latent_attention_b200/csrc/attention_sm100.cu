@@ -110,6 +110,10 @@ enum : int { kSplitPublish = 1, kSplitMerge = 2, kSplitAbort = 3 };  // split ha
 #define SD_PING_RELEASE -1  // tuning override of Cfg::PING_RELEASE (-1: the per-config choice)
 #endif
 
+#ifndef SD_MMA_BLOCKING
+#define SD_MMA_BLOCKING 0  // MMA issuers in a fixed order behind suspending waits instead of polling
+#endif
+
 #ifndef SD_EXP_SPLIT
 #define SD_EXP_SPLIT 1  // special-function pairs before the token hand-off, polynomial pairs after
 #endif
@@ -419,6 +423,52 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       bool ok = true;
       long long t_idle = clock64();
       uint32_t spins = 0;
+      // Blocking variant: the fixed order S_0, then S_{g+1} (the softmax releases S_g right after
+      // reading it) before P_g V_g, each behind suspending mbarrier waits instead of polling, so an
+      // idle issuer takes no issue slots from the softmax warps of its sub-partition.
+      constexpr bool kBlocking = SD_MMA_BLOCKING && C::P_SEP;
+      if constexpr (kBlocking) {
+        auto do_qk = [&]() -> bool {
+          const int qb = nseg_q % C::QBUF;
+          if (jq == 0 && !wait_bar(bars.q_full(qb), (nseg_q / C::QBUF) & 1, abort_flag, err)) return false;
+          if (!wait_bar(bars.k_full(gq % STAGES), (gq / STAGES) & 1, abort_flag, err)) return false;
+          if (gq > 0 && !wait_bar(bars.s_free(t), (gq - 1) & 1, abort_flag, err)) return false;
+          tc_fence_after();
+          tq = sbase + C::Q_OFF + (qb * NQ + t) * C::Q_TILE_BYTES;
+          issue_qk(gq % STAGES);
+          mma_commit(bars.s_full(t));
+          ++gq;
+          if (++jq == sq.ke - sq.kb) {
+            mma_commit(bars.q_empty(qb));
+            have_q = next_seg(uq, u1, nkv, sq);
+            jq = 0;
+            ++nseg_q;
+          }
+          return true;
+        };
+        auto do_pv = [&]() -> bool {
+          if (!wait_bar(bars.p_full(t), gp & 1, abort_flag, err)) return false;
+          if (!wait_bar(C::L_IN_V ? bars.v_ready(gp % STAGES) : bars.v_full(gp % STAGES), (gp / STAGES) & 1,
+                        abort_flag, err))
+            return false;
+          tc_fence_after();
+          issue_pv(gp % STAGES, jp == 0);
+          mma_commit(bars.o_done(t));
+          mma_commit(bars.kv_empty(gp % STAGES));
+          ++gp;
+          if (++jp == sp.ke - sp.kb) {
+            have_p = next_seg(up, u1, nkv, sp);
+            jp = 0;
+          }
+          return true;
+        };
+        if (have_q) ok = do_qk();
+        while (ok && have_p) {
+          if (have_q && !do_qk()) break;
+          if (!do_pv()) break;
+        }
+        have_p = false;
+      }
       while (ok && have_p) {
         const bool can_pv = gp < gq && mbar_test_wait(bars.p_full(t), gp & 1) &&
                             mbar_test_wait(C::L_IN_V ? bars.v_ready(gp % STAGES) : bars.v_full(gp % STAGES),
