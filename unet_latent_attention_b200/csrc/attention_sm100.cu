@@ -110,6 +110,10 @@ enum : int { kSplitPublish = 1, kSplitMerge = 2, kSplitAbort = 3 };  // split ha
 #define SD_PING_RELEASE -1  // tuning override of Cfg::PING_RELEASE (-1: the per-config choice)
 #endif
 
+#ifndef SD_REGSPLIT
+#define SD_REGSPLIT 0  // setmaxnreg: 56 registers per helper thread, 224 per softmax thread
+#endif
+
 #ifndef SD_MMA_BLOCKING
 #define SD_MMA_BLOCKING 0  // MMA issuers in a fixed order behind suspending waits instead of polling
 #endif
@@ -192,6 +196,10 @@ struct Cfg {
   static constexpr int SOFT_WARP0 = 4;
   static constexpr int NUM_WARPS = 4 + 4 * NQ;
   static constexpr int THREADS = 32 * NUM_WARPS;
+  // Register split (setmaxnreg) for NQ = 2: the helper warpgroup drops to REG_HELPER per thread and
+  // the two softmax warpgroups rise to REG_SOFT, within the launch's 384 x 168.
+  static constexpr int REG_HELPER = 56, REG_SOFT = 224;
+  static_assert(NQ != 2 || 128 * REG_HELPER + 256 * REG_SOFT <= 168 * 384, "register split exceeds the launch budget");
   // Split-item hand-off slot: raw O (NPV fp32 per row) and (m, l) per row of the NQ tiles.
   static constexpr int SLOT_FLOATS = NQ * BM * (NPV + 2);
   // Column pairs after which a softmax warp passes the ping-pong token (measured: half-way for
@@ -326,6 +334,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   if (warp < C::SOFT_WARP0) {
   // ==================================================================== helper warpgroup
+  if constexpr (SD_REGSPLIT && NQ == 2) regs_dec<C::REG_HELPER>();  // registers move to the softmax warpgroups
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -547,6 +556,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   }
   } else {
   // ==================================================================== softmax warpgroups
+  if constexpr (SD_REGSPLIT && NQ == 2) regs_inc<C::REG_SOFT>();
   {
     // ------------------------------------------------------------------ softmax warps
     const int t = (warp - C::SOFT_WARP0) >> 2;  // query tile of this warpgroup
