@@ -140,6 +140,17 @@ def test_split_items_either_piece_may_merge(cuda, dh, heads, Lq, Lk):
     _check(reversed_.float().cpu().numpy(), oracle.attention(q, k, v))
 
 
+def test_split_items_after_other_head_dims(cuda):
+    # every head dim's launches share one hand-off workspace; each must leave the counters at zero
+    # and find them at zero whatever configuration ran before it (the slots of one configuration
+    # must never lie where another expects its counters)
+    for dh, heads, Lq, Lk in [(64, 80, 256, 1000), (40, 80, 256, 640), (80, 80, 256, 700), (160, 120, 128, 300),
+                              (40, 96, 300, 129), (64, 80, 256, 1000)]:
+        q, k, v = _qkv(2, heads, Lq, Lk, dh, 9400 + dh + Lk)
+        o = _run(q, k, v, cuda)
+        _check(o, oracle.attention(q, k, v))
+
+
 def test_repeated_launches_reuse_the_hand_off_flags(cuda):
     # the split hand-off flags must return to zero after every launch (graph replays rely on it)
     q, k, v = _qkv(2, 80, 256, 640, 40, 9100)

@@ -119,7 +119,7 @@ enum : int { kSplitPublish = 1, kSplitMerge = 2, kSplitAbort = 3 };  // split ha
 #endif
 
 #ifndef SD_EXP_SPLIT
-#define SD_EXP_SPLIT 1  // special-function pairs before the token hand-off, polynomial pairs after
+#define SD_EXP_SPLIT 0  // 1: special-function pairs before the token hand-off, polynomial pairs after (slower)
 #endif
 
 #ifndef SD_PINGPONG
@@ -252,6 +252,7 @@ struct Seg {
 // Unit ranges of the persistent grid: CTA c owns units [u[c], u[c+1]). Passed by value (kernel
 // parameter space), filled on the host: evenly, or balanced by a cost model (see part_ranges).
 constexpr int kMaxCtas = 256;
+constexpr size_t kCounterBytes = kMaxCtas * sizeof(unsigned int);  // split-item counters, workspace head
 struct Part {
   long long u[kMaxCtas + 1];
 };
@@ -1098,8 +1099,10 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
   float* ws = nullptr;
   unsigned int* flags = nullptr;
   if (G < items && nkv > 1) {
-    const size_t fbytes = (static_cast<size_t>(G) * C::SLOT_FLOATS * sizeof(float) + 255) / 256 * 256;
-    const size_t need = fbytes + static_cast<size_t>(G) * sizeof(unsigned int);
+    // Layout: the boundary counters first, at the same place for every configuration (a launch of
+    // one head dim must never find another configuration's slot data where it expects counters
+    // that the previous launches left at zero), then the slots.
+    const size_t need = kCounterBytes + static_cast<size_t>(G) * C::SLOT_FLOATS * sizeof(float);
     void* p = nullptr;
     if (fixed) {
       if (need > kFixedScratchBytes)
@@ -1107,14 +1110,13 @@ sd_status launch(const void* q, const void* k, const void* v, void* o, int64_t B
                                             "buffer holds %zu", need, kFixedScratchBytes);
       st = fixed_scratch(&p);
       if (st != SD_OK) return st;
-      st = sd::cuda_check(cudaMemsetAsync(static_cast<char*>(p) + fbytes, 0, need - fbytes, s),
-                          "cudaMemsetAsync(fixed scratch flags)");
+      st = sd::cuda_check(cudaMemsetAsync(p, 0, kCounterBytes, s), "cudaMemsetAsync(fixed scratch counters)");
     } else {
       st = workspace(need, s, &p);
     }
     if (st != SD_OK) return st;
-    ws = static_cast<float*>(p);
-    flags = reinterpret_cast<unsigned int*>(static_cast<char*>(p) + fbytes);
+    flags = static_cast<unsigned int*>(p);
+    ws = reinterpret_cast<float*>(static_cast<char*>(p) + kCounterBytes);
   }
   Part part;
   part_ranges(items * nkv, nkv, static_cast<int>(G), CostModel{C::COST_SEG, C::COST_TAIL, C::COST_HEAD}, part.u);

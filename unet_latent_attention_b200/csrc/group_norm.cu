@@ -41,7 +41,7 @@ constexpr int kMaxItems = 16;  // float4 per thread on the resident path
 #define SD_GN_POLICY 0
 #endif
 #ifndef SD_GN_PERSIST
-#define SD_GN_PERSIST 1  // the persistent two-groups-in-flight path where it applies
+#define SD_GN_PERSIST 0  // 1: the persistent two-groups-in-flight path where it applies (measured slower)
 #endif
 #ifndef SD_GN_GPC
 #define SD_GN_GPC 2  // groups per cluster of the persistent path (fewer clusters when fewer fit)
