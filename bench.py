@@ -576,37 +576,81 @@ def bench_extra(sdk, dev, hbm):
 
 
 def bench_e2e(args, sdk, S, g, a_t, a_p, w, flops_step, world, dev):
-    """Same step through the public API with host buffers: pinned H2D of every input, the four
-    launches, D2H of every output, all inside the timed region."""
+    """Same step through the public API with host buffers: every step copies all of its inputs from
+    pinned host memory to the device, runs the four launches and copies every output back, all inside
+    the timed region. Two device buffer sets and three streams let step i's inputs travel while step
+    i-1 computes and step i-2's outputs travel back (the host link carries both directions at once);
+    the serial form (one stream) is reported beside it."""
     import torch
     host_in = {k: S[k].cpu().pin_memory() for k in INPUT_KEYS}
     host_out = {k: torch.empty(S[k].shape, dtype=S[k].dtype, pin_memory=True) for k in OUTPUT_KEYS}
-    dev_buf = {k: torch.empty_like(S[k]) for k in INPUT_KEYS + OUTPUT_KEYS}
+    bufs = [{k: torch.empty_like(S[k]) for k in INPUT_KEYS + OUTPUT_KEYS} for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
     n = max(3, min(args.steps, 50))
+    s_in, s_c, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
 
-    def one():
-        for k in INPUT_KEYS:
-            dev_buf[k].copy_(host_in[k], non_blocking=True)
-        run_step(sdk, dev_buf, g, a_t, a_p, w)
-        for k in OUTPUT_KEYS:
-            host_out[k].copy_(dev_buf[k], non_blocking=True)
+    def pipelined(steps, e0=None, e1=None):
+        ev_in = [torch.cuda.Event() for _ in range(steps)]
+        ev_c = [torch.cuda.Event() for _ in range(steps)]
+        ev_out = [torch.cuda.Event() for _ in range(steps)]
+        if e0 is not None:
+            e0.record(s_in)
+        for i in range(steps):
+            b = bufs[i % 2]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_c[i - 2])  # step i-2 has finished reading this set's inputs
+                for k in INPUT_KEYS:
+                    b[k].copy_(host_in[k], non_blocking=True)
+                ev_in[i].record(s_in)
+            with torch.cuda.stream(s_c):
+                s_c.wait_event(ev_in[i])
+                if i >= 2:
+                    s_c.wait_event(ev_out[i - 2])  # step i-2's outputs have left this set
+                run_step(sdk, b, g, a_t, a_p, w)
+                ev_c[i].record(s_c)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_c[i])
+                for k in OUTPUT_KEYS:
+                    host_out[k].copy_(b[k], non_blocking=True)
+                ev_out[i].record(s_out)
+        if e1 is not None:
+            s_out.wait_event(ev_out[-1])
+            e1.record(s_out)
 
-    for _ in range(3):
-        one()
+    def serial(steps):
+        b = bufs[0]
+        for _ in range(steps):
+            for k in INPUT_KEYS:
+                b[k].copy_(host_in[k], non_blocking=True)
+            run_step(sdk, b, g, a_t, a_p, w)
+            for k in OUTPUT_KEYS:
+                host_out[k].copy_(b[k], non_blocking=True)
+
+    pipelined(3)
+    serial(3)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(n):
-        one()
-    e1.record()
+    pipelined(n, e0, e1)
     torch.cuda.synchronize()
     ms = reduce_max([e0.elapsed_time(e1)], dev)[0]
+    if world > 1:
+        torch.distributed.barrier()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record()
+    serial(n)
+    f1.record()
+    torch.cuda.synchronize()
+    ms_serial = reduce_max([f0.elapsed_time(f1)], dev)[0]
+    sdk.sd_device_status()
     return {"value": whole_job_tflops(flops_step, n, world, ms), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms / n, "steps": n}
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms / n, "steps": n,
+            "form": "two buffer sets, copy-in / compute / copy-out streams",
+            "serial": {"value": whole_job_tflops(flops_step, n, world, ms_serial), "ms_per_step": ms_serial / n}}
 
 
 # -------------------------------------------------------------------------------- CPU oracle arm
