@@ -40,12 +40,7 @@ constexpr int kMaxItems = 16;  // float4 per thread on the resident path
 #ifndef SD_GN_POLICY
 #define SD_GN_POLICY 0
 #endif
-#ifndef SD_GN_PERSIST
-#define SD_GN_PERSIST 0  // 1: the persistent two-groups-in-flight path where it applies (measured slower)
-#endif
-#ifndef SD_GN_GPC
-#define SD_GN_GPC 2  // groups per cluster of the persistent path (fewer clusters when fewer fit)
-#endif
+
 
 struct Stats {
   float n, mean, m2;
@@ -219,89 +214,6 @@ __global__ void __launch_bounds__(THREADS, (SD_GN_MINB && THREADS == 512 && ITEM
   }
 }
 
-// Persistent path: cluster k of n_cl clusters of `cs` CTAs takes the groups k, k + n_cl, ...; CTA
-// `rank` owns elements [rank*chunk, (rank+1)*chunk) of each. A thread holds its part of two groups
-// in registers: the loads of the next group are in flight while the current group's statistics
-// are merged over the cluster and its output is written, so reads and writes overlap instead of
-// all reads of a launch preceding all of its writes. The cluster-wide slots are double-buffered by
-// group parity (a slow CTA may still read one group's slots while its peers fill the next ones).
-template <int ITEMS, int THREADS, int EPI>
-__global__ void __launch_bounds__(THREADS, 1) gn_persistent(const float* x, const float* __restrict__ gamma,
-                                                           const float* __restrict__ beta, void* y, int group_elems,
-                                                           int chunk, int hw, int cpg, int groups, int n_groups,
-                                                           float eps) {
-  __shared__ Stats s_warp[THREADS / 32];
-  __shared__ Stats s_all[2][kMaxCluster];
-  __shared__ float s_mr[2][2];
-  sd::grid_dep_wait();
-  sd::grid_dep_launch();
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = static_cast<int>(cluster.block_rank());
-  const int cs = static_cast<int>(cluster.num_blocks());
-  const int cl = blockIdx.x / cs, n_cl = gridDim.x / cs;
-  const int n4 = chunk >> 2;
-  const int e0 = rank * chunk;
-
-  auto load = [&](float4 (&v)[ITEMS], int grp) {
-    const float4* xg = reinterpret_cast<const float4*>(x + static_cast<int64_t>(grp) * group_elems + e0);
-#pragma unroll
-    for (int i = 0; i < ITEMS; ++i) {
-      const int idx = threadIdx.x + i * THREADS;
-      v[i] = idx < n4 ? ld_stream(xg + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  };
-  auto process = [&](const float4 (&v)[ITEMS], int grp, int par) {
-    float sum = 0.f, cnt = 0.f;
-#pragma unroll
-    for (int i = 0; i < ITEMS; ++i) {
-      if (threadIdx.x + i * THREADS < n4) {
-        sum += (v[i].x + v[i].y) + (v[i].z + v[i].w);
-        cnt += 4.f;
-      }
-    }
-    Stats st{cnt, cnt > 0.f ? sum / cnt : 0.f, 0.f};
-#pragma unroll
-    for (int i = 0; i < ITEMS; ++i) {
-      if (threadIdx.x + i * THREADS < n4) {
-        const float a = v[i].x - st.mean, b = v[i].y - st.mean, c = v[i].z - st.mean, d = v[i].w - st.mean;
-        st.m2 += a * a + b * b + c * c + d * d;
-      }
-    }
-    cluster_group_stats(st, eps, &s_mr[par][0], &s_mr[par][1], s_warp, s_all[par]);
-    const float mean = s_mr[par][0], rstd = s_mr[par][1];
-    const int g = grp % groups;
-    const int64_t base4 = (static_cast<int64_t>(grp) * group_elems + e0) >> 2;
-#pragma unroll
-    for (int i = 0; i < ITEMS; ++i) {
-      const int idx = threadIdx.x + i * THREADS;
-      if (idx < n4) {
-        const int c = g * cpg + (e0 + idx * 4) / hw;  // hw % 4 == 0: a float4 never straddles channels
-        const float a = rstd * __ldg(gamma + c);
-        const float b = fmaf(-mean, a, __ldg(beta + c));
-        store4<EPI>(y, base4 + idx, make_float4(fmaf(v[i].x, a, b), fmaf(v[i].y, a, b), fmaf(v[i].z, a, b),
-                                                fmaf(v[i].w, a, b)));
-      }
-    }
-  };
-
-  float4 va[ITEMS], vb[ITEMS];
-  int g = cl, par = 0;
-  if (g < n_groups) load(va, g);
-  while (g < n_groups) {
-    int gn = g + n_cl;
-    if (gn < n_groups) load(vb, gn);
-    process(va, g, par);
-    par ^= 1;
-    g = gn;
-    if (g >= n_groups) break;
-    gn = g + n_cl;
-    if (gn < n_groups) load(va, gn);
-    process(vb, g, par);
-    par ^= 1;
-    g = gn;
-  }
-}
-
 // Streaming path: any shape and alignment. CTA `rank` of the cluster owns elements [lo, hi) of the
 // group; sweep 1 builds the triple (exact stats of each run of four values, merged pairwise),
 // sweep 2 normalises.
@@ -373,33 +285,6 @@ cudaError_t launch_resident(dim3 grid, int cs, cudaStream_t s, const float* x, c
                             groups, eps);
 }
 
-template <int ITEMS, int THREADS, int EPI>
-cudaError_t launch_persistent(int cs, int64_t n_groups, cudaStream_t s, const float* x, const float* gamma,
-                              const float* beta, void* y, int group_elems, int chunk, int hw, int cpg, int groups,
-                              float eps) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(THREADS);
-  cfg.stream = s;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  // Clusters: about SD_GN_GPC groups each, at most as many as can be resident at once.
-  auto kern = gn_persistent<ITEMS, THREADS, EPI>;
-  int max_cl = 0;
-  cfg.gridDim = dim3(static_cast<unsigned>(cs));
-  if (cudaOccupancyMaxActiveClusters(&max_cl, kern, &cfg) != cudaSuccess || max_cl < 1) max_cl = 1;
-  int64_t n_cl = (n_groups + SD_GN_GPC - 1) / SD_GN_GPC;
-  if (n_cl > max_cl) n_cl = max_cl;
-  cfg.gridDim = dim3(static_cast<unsigned>(n_cl * cs));
-  cfg.numAttrs = 1 + sd::pdl_attr(&attr[1]);
-  return cudaLaunchKernelEx(&cfg, kern, x, gamma, beta, y, group_elems, chunk, hw, cpg, groups,
-                            static_cast<int>(n_groups), eps);
-}
-
 // One GroupNorm launch with epilogue EPI; `name` prefixes error messages.
 template <int EPI>
 sd_status group_norm_impl(const char* name, const float* x, const float* gamma, const float* beta, void* y, int64_t B,
@@ -464,31 +349,6 @@ sd_status group_norm_impl(const char* name, const float* x, const float* gamma, 
     }
   }
   cudaError_t err;
-  // Persistent path: 256- or 512-thread CTAs in the smallest cluster that holds a group's part in at
-  // most 8 float4 per thread (two groups in flight), when there are at least two groups per cluster.
-  int pcs = 0, pth = 0;
-  if (vec_ok && SD_GN_PERSIST) {
-    for (int th = 256; th <= 512 && !pcs; th *= 2)
-      for (int c = 1; c <= kMaxCluster && !pcs; c *= 2)
-        if (group_elems % (4 * c) == 0 && group_elems / c <= int64_t(th) * 4 * 8) {
-          pcs = c;
-          pth = th;
-        }
-    if (pcs && n_groups < 2 * SD_GN_GPC) pcs = 0;
-  }
-  if (pcs > 0) {
-    const int chunk = static_cast<int>(group_elems / pcs);
-    const int need = (chunk / 4 + pth - 1) / pth;
-    const int ge = static_cast<int>(group_elems), ihw = static_cast<int>(hw), icpg = static_cast<int>(cpg),
-              ig = static_cast<int>(groups);
-#define SD_GN_PCASE(N, T) \
-  if (pth == T && need <= N) err = launch_persistent<N, T, EPI>(pcs, n_groups, s, x, gamma, beta, y, ge, chunk, ihw, icpg, ig, eps); else
-    SD_GN_PCASE(1, 256) SD_GN_PCASE(2, 256) SD_GN_PCASE(3, 256) SD_GN_PCASE(4, 256) SD_GN_PCASE(5, 256)
-    SD_GN_PCASE(6, 256) SD_GN_PCASE(8, 256) SD_GN_PCASE(5, 512) SD_GN_PCASE(6, 512) SD_GN_PCASE(8, 512)
-    err = cudaErrorInvalidValue;
-#undef SD_GN_PCASE
-    return sd::cuda_check(err, "group norm launch");
-  }
   if (cs > 0) {
     const int chunk = static_cast<int>(group_elems / cs);
     const int need = (chunk / 4 + threads - 1) / threads;
