@@ -37,7 +37,7 @@ WID = 2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
 ATTN_SOURCES = ["unet_latent_attention_b200/csrc/attention_sm100.cu", "unet_latent_attention_b200/csrc/sm100_ptx.cuh",
-                "unet_latent_attention_b200/csrc/sd_internal.h"]
+                "unet_latent_attention_b200/csrc/sd_internal.h", "unet_latent_attention_b200/csrc/attn_common.cuh"]
 TRAFFIC_FILE = "profiles/attention_self_sd15_512.md"
 
 
