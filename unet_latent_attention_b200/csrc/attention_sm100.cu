@@ -110,6 +110,10 @@ enum : int { kSplitPublish = 1, kSplitMerge = 2, kSplitAbort = 3 };  // split ha
 #define SD_PING_RELEASE -1  // tuning override of Cfg::PING_RELEASE (-1: the per-config choice)
 #endif
 
+#ifndef SD_SOFTMAX_STREAM
+#define SD_SOFTMAX_STREAM 0  // read S from tensor memory twice in 64-column halves instead of holding it whole
+#endif
+
 #ifndef SD_REGSPLIT
 #define SD_REGSPLIT 0  // setmaxnreg: 56 registers per helper thread, 224 per softmax thread
 #endif
@@ -582,6 +586,113 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         break;
       }
       tc_fence_after();
+      // Streaming variant: S is read from tensor memory twice (once for the row max, once for the
+      // exponentials), 64 columns at a time, instead of being held whole in registers; P goes to
+      // tensor memory 32 packed columns at a time. S is released after the second read.
+      constexpr bool kStream = SD_SOFTMAX_STREAM && C::P_SEP && BN == 128;
+      if constexpr (kStream) {
+        const int valid = Lk - j * BN;
+        auto load64 = [&](int h, float (&v)[64]) {
+          uint32_t ra[32], rb[32];
+          tmem_ld32(tS + h * 64, ra);
+          tmem_ld32(tS + h * 64 + 32, rb);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            v[i] = __uint_as_float(ra[i]);
+            v[32 + i] = __uint_as_float(rb[i]);
+          }
+          if (valid < BN) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              if (h * 64 + i >= valid) v[i] = -INFINITY;
+          }
+        };
+        float pm[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) pm[k] = -INFINITY;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float v[64];
+          load64(h, v);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            pm[k] = max3f(pm[k], v[k], v[16 + k]);
+            pm[k] = max3f(pm[k], v[32 + k], v[48 + k]);
+          }
+        }
+        const float mx = fmaxf(max3f(max3f(pm[0], pm[1], pm[2]), max3f(pm[3], pm[4], pm[5]), max3f(pm[6], pm[7], pm[8])),
+                               max3f(max3f(pm[9], pm[10], pm[11]), max3f(pm[12], pm[13], pm[14]), pm[15]));
+        const float m_new = fmaxf(m_run, mx * scale_log2);
+        const bool rescale = __any_sync(0xffffffffu, m_new > m_run + 8.0f);
+        const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
+        if (rescale) m_run = m_new;
+        // P is written as it is produced: the previous P V must be complete (and O rescaled) first
+        if (gi > 0) {
+          if (!__all_sync(0xffffffffu, wait_bar(bars.o_done(t), (gi - 1) & 1, abort_flag, err))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        if (rescale && !first) {
+#pragma unroll
+          for (int c = 0; c < C::NPV / 16; ++c) {
+            uint32_t r[16];
+            tmem_ld16(tO + c * 16, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st16(tO + c * 16, r);
+          }
+        }
+        if (kPing && (t == 1 || gi > 0)) {
+          if (!__all_sync(0xffffffffu, wait_bar(bars.tok(t, quarter), (t == 1 ? gi : gi - 1) & 1, abort_flag, err))) {
+            ok = false;
+            break;
+          }
+        }
+        const float neg_m = -m_run;
+        float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float v[64];
+          load64(h, v);
+          uint32_t pk[32];
+#pragma unroll
+          for (int b = 0; b < 32; ++b) {
+            float x0, x1;
+            fma2(x0, x1, v[2 * b], v[2 * b + 1], scale_log2, scale_log2, neg_m, neg_m);
+            if ((b & 7) < C::POLY_PAIRS) {
+              exp2_poly2(x0, x1, x0, x1);
+            } else {
+              x0 = ex2_approx(x0);
+              x1 = ex2_approx(x1);
+            }
+            if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x0, x1);
+            pk[b] = C::F16 ? pack_f16x2(x0, x1) : pack_bf16x2(x0, x1);
+          }
+          uint32_t r0[16], r1[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            r0[i] = pk[i];
+            r1[i] = pk[16 + i];
+          }
+          tmem_st16(tP + h * 32, r0);
+          tmem_st16(tP + h * 32 + 16, r1);
+        }
+        if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
+        if (kPing) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
+        }
+        tc_fence_before();
+        mbar_arrive(bars.s_free(t));  // both reads of S are complete (tcgen05.wait::ld above)
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bars.p_full(t));
+        continue;
+      }
       float sv[BN];
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
