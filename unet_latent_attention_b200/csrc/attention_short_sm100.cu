@@ -122,8 +122,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // this CTA's tiles [t0, t0 + n): an equal share of the tile list
   const long long t0 = n_tiles * blockIdx.x / gridDim.x;
   const int n = static_cast<int>(n_tiles * (blockIdx.x + 1) / gridDim.x - t0);
-  auto head_of = [&](int i) { return static_cast<int>((t0 + i) / tiles_per_head); };
-  auto row0_of = [&](int i) { return static_cast<int>((t0 + i) % tiles_per_head) * BM; };
+  // Plane and first query row of local tile i. One 64-bit division at entry; 32-bit arithmetic after
+  // (a 64-bit division is a long software routine, and these run once per tile in every role).
+  const unsigned tph = static_cast<unsigned>(tiles_per_head);
+  const int bh0 = static_cast<int>(t0 / tiles_per_head);
+  const unsigned qt0 = static_cast<unsigned>(t0 - static_cast<long long>(bh0) * tiles_per_head);
+  auto head_of = [&](int i) { return bh0 + static_cast<int>((qt0 + static_cast<unsigned>(i)) / tph); };
+  auto row0_of = [&](int i) { return static_cast<int>((qt0 + static_cast<unsigned>(i)) % tph) * BM; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < QS; ++i) {
