@@ -98,12 +98,6 @@ struct ShortBars {
   __device__ uint32_t fin() const { return base + 8 * (2 * C::QS + 4 * C::KVB + 4 * C::NSLOT); }
 };
 
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
-               :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-               : "memory");
-}
-
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_short_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,

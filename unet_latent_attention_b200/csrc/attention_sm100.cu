@@ -110,10 +110,6 @@ enum : int { kSplitPublish = 1, kSplitMerge = 2, kSplitAbort = 3 };  // split ha
 #define SD_PING_RELEASE -1  // tuning override of Cfg::PING_RELEASE (-1: the per-config choice)
 #endif
 
-#ifndef SD_SOFTMAX_STREAM
-#define SD_SOFTMAX_STREAM 0  // read S from tensor memory twice in 64-column halves instead of holding it whole
-#endif
-
 #ifndef SD_REGSPLIT
 #define SD_REGSPLIT 0  // setmaxnreg: 56 registers per helper thread, 224 per softmax thread
 #endif
@@ -179,9 +175,9 @@ struct Cfg {
   static constexpr int V_OFF = K_OFF + STAGES * K_TILE_BYTES;
   static constexpr int BAR_OFF = V_OFF + STAGES * V_TILE_BYTES;
   // q_full, k_full[S], v_full[S], v_ready[S], kv_empty[S], s_full[NQ], s_free[NQ], p_full[NQ], o_done[NQ],
-  // fin[NQ], the exp tokens tok[2][4] of the two tiles' warps on each SM sub-partition, q_empty[2],
+  // fin[NQ], the exp tokens tok[NQ][4] of the tiles' warps on each SM sub-partition, q_empty[2],
   // split_dec[2], split_written[2]
-  static constexpr int NBARS = 2 + 4 * STAGES + 5 * NQ + 8 + 2 + 4;
+  static constexpr int NBARS = 2 + 4 * STAGES + 9 * NQ + 2 + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   // misc: TMEM base address, abort flag, the split hand-off decisions of the two piece kinds
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
@@ -237,11 +233,11 @@ struct Bars {
   __device__ uint32_t o_done(int t) const { return base + 8 * (2 + 4 * stages + 3 * nq + t); }
   __device__ uint32_t fin() const { return base + 8 * (2 + 4 * stages + 4 * nq); }
   __device__ uint32_t tok(int t, int q) const { return base + 8 * (2 + 4 * stages + 5 * nq + 4 * t + q); }
-  __device__ uint32_t q_empty(int b) const { return base + 8 * (2 + 4 * stages + 5 * nq + 8 + b); }
+  __device__ uint32_t q_empty(int b) const { return base + 8 * (2 + 4 * stages + 9 * nq + b); }
   // split-item hand-off of the tail piece (kind 0) and the head piece (kind 1): the leader's
   // decision is published, and this piece's slot has been written by every softmax thread
-  __device__ uint32_t split_dec(int kind) const { return base + 8 * (2 + 4 * stages + 5 * nq + 10 + kind); }
-  __device__ uint32_t split_written(int kind) const { return base + 8 * (2 + 4 * stages + 5 * nq + 12 + kind); }
+  __device__ uint32_t split_dec(int kind) const { return base + 8 * (2 + 4 * stages + 9 * nq + 2 + kind); }
+  __device__ uint32_t split_written(int kind) const { return base + 8 * (2 + 4 * stages + 9 * nq + 4 + kind); }
 };
 
 // Persistent schedule: the work is items x nkv units (an item = NQ query tiles of one (b, h); a
@@ -309,7 +305,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_init(bars.o_done(t), 1);
     }
     for (int t = 0; t < NQ; ++t) mbar_init(bars.fin() + 8 * t, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(bars.tok(i >> 2, i & 3), 1);
+    for (int i = 0; i < 4 * NQ; ++i) mbar_init(bars.tok(i >> 2, i & 3), 1);
     mbar_init(bars.q_empty(0), NQ);
     mbar_init(bars.q_empty(1), NQ);
     for (int kind = 0; kind < 2; ++kind) {
@@ -570,7 +566,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const uint32_t tbase = tmem + t * C::TM_TILE + (static_cast<uint32_t>(quarter * 32) << 16);
     const uint32_t tS = tbase + C::TM_S, tP = tbase + C::TM_P, tO = tbase + C::TM_O;
     bool ok = true;
-    constexpr bool kPing = SD_PINGPONG && NQ == 2 && (SD_PING_SHORT || BN == 128);
+    constexpr bool kPing = SD_PINGPONG && NQ >= 2 && (SD_PING_SHORT || BN == 128);
     long long u = u0;
     Seg sg;
     int gi = 0;  // CTA-wide K/V tile count: the phase of every per-tile barrier
@@ -586,113 +582,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         break;
       }
       tc_fence_after();
-      // Streaming variant: S is read from tensor memory twice (once for the row max, once for the
-      // exponentials), 64 columns at a time, instead of being held whole in registers; P goes to
-      // tensor memory 32 packed columns at a time. S is released after the second read.
-      constexpr bool kStream = SD_SOFTMAX_STREAM && C::P_SEP && BN == 128;
-      if constexpr (kStream) {
-        const int valid = Lk - j * BN;
-        auto load64 = [&](int h, float (&v)[64]) {
-          uint32_t ra[32], rb[32];
-          tmem_ld32(tS + h * 64, ra);
-          tmem_ld32(tS + h * 64 + 32, rb);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            v[i] = __uint_as_float(ra[i]);
-            v[32 + i] = __uint_as_float(rb[i]);
-          }
-          if (valid < BN) {
-#pragma unroll
-            for (int i = 0; i < 64; ++i)
-              if (h * 64 + i >= valid) v[i] = -INFINITY;
-          }
-        };
-        float pm[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) pm[k] = -INFINITY;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float v[64];
-          load64(h, v);
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            pm[k] = max3f(pm[k], v[k], v[16 + k]);
-            pm[k] = max3f(pm[k], v[32 + k], v[48 + k]);
-          }
-        }
-        const float mx = fmaxf(max3f(max3f(pm[0], pm[1], pm[2]), max3f(pm[3], pm[4], pm[5]), max3f(pm[6], pm[7], pm[8])),
-                               max3f(max3f(pm[9], pm[10], pm[11]), max3f(pm[12], pm[13], pm[14]), pm[15]));
-        const float m_new = fmaxf(m_run, mx * scale_log2);
-        const bool rescale = __any_sync(0xffffffffu, m_new > m_run + 8.0f);
-        const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.0f;
-        if (rescale) m_run = m_new;
-        // P is written as it is produced: the previous P V must be complete (and O rescaled) first
-        if (gi > 0) {
-          if (!__all_sync(0xffffffffu, wait_bar(bars.o_done(t), (gi - 1) & 1, abort_flag, err))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-        }
-        if (rescale && !first) {
-#pragma unroll
-          for (int c = 0; c < C::NPV / 16; ++c) {
-            uint32_t r[16];
-            tmem_ld16(tO + c * 16, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st16(tO + c * 16, r);
-          }
-        }
-        if (kPing && (t == 1 || gi > 0)) {
-          if (!__all_sync(0xffffffffu, wait_bar(bars.tok(t, quarter), (t == 1 ? gi : gi - 1) & 1, abort_flag, err))) {
-            ok = false;
-            break;
-          }
-        }
-        const float neg_m = -m_run;
-        float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float v[64];
-          load64(h, v);
-          uint32_t pk[32];
-#pragma unroll
-          for (int b = 0; b < 32; ++b) {
-            float x0, x1;
-            fma2(x0, x1, v[2 * b], v[2 * b + 1], scale_log2, scale_log2, neg_m, neg_m);
-            if ((b & 7) < C::POLY_PAIRS) {
-              exp2_poly2(x0, x1, x0, x1);
-            } else {
-              x0 = ex2_approx(x0);
-              x1 = ex2_approx(x1);
-            }
-            if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x0, x1);
-            pk[b] = C::F16 ? pack_f16x2(x0, x1) : pack_bf16x2(x0, x1);
-          }
-          uint32_t r0[16], r1[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            r0[i] = pk[i];
-            r1[i] = pk[16 + i];
-          }
-          tmem_st16(tP + h * 32, r0);
-          tmem_st16(tP + h * 32 + 16, r1);
-        }
-        if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
-        if (kPing) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
-        }
-        tc_fence_before();
-        mbar_arrive(bars.s_free(t));  // both reads of S are complete (tcgen05.wait::ld above)
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bars.p_full(t));
-        continue;
-      }
       float sv[BN];
 #pragma unroll
       for (int c = 0; c < BN / 32; ++c) {
@@ -760,8 +649,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // Ping-pong: the special-function unit of a sub-partition serves one tile's exp2 phase at a
       // time; the other tile's warp on it does its row max, P store and S load meanwhile. Tile 0
       // goes first; each warp hands the token to its partner (same sub-partition) after its exps.
-      if (kPing && (t == 1 || gi > 0)) {
-        if (!__all_sync(0xffffffffu, wait_bar(bars.tok(t, quarter), (t == 1 ? gi : gi - 1) & 1, abort_flag, err))) {
+      if (kPing && (t > 0 || gi > 0)) {
+        if (!__all_sync(0xffffffffu, wait_bar(bars.tok(t, quarter), (t > 0 ? gi : gi - 1) & 1, abort_flag, err))) {
           ok = false;
           break;
         }
@@ -793,7 +682,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           pk[b] = C::F16 ? pack_f16x2(x0, x1) : pack_bf16x2(x0, x1);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
+        if (lane == 0) mbar_arrive(bars.tok(t + 1 == NQ ? 0 : t + 1, quarter));
 #pragma unroll
         for (int b = 0; b < BN / 2; ++b) {
           if ((b & 7) >= C::POLY_PAIRS) continue;
@@ -808,7 +697,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int b = 0; b < BN / 2 && !kSplit; b += EB) {
         if (kPing && kRelease < BN / 2 && b == kRelease) {
           __syncwarp();
-          if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
+          if (lane == 0) mbar_arrive(bars.tok(t + 1 == NQ ? 0 : t + 1, quarter));
         }
         float x[2 * EB];
 #pragma unroll
@@ -839,7 +728,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
       if (kPing && kRelease == BN / 2 && !kSplit) {
         __syncwarp();
-        if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
+        if (lane == 0) mbar_arrive(bars.tok(t + 1 == NQ ? 0 : t + 1, quarter));
       }
       // The previous P V (and the O it accumulates) must be complete before P and O are touched.
       if (!kChunkP && C::P_SEP && gi > 0) {
