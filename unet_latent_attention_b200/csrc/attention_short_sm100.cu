@@ -17,8 +17,8 @@
 //    O = P V once the softmax has written P over S in the same slot (the "A in TMEM" form). The row
 //    sums come out of P V through a column of ones written into V (column dh).
 //  * Two softmax warpgroups take alternate tiles: tcgen05.ld of the 80 scores, row max, exp2,
-//    tcgen05.st of P; then, while the next tile's P V runs, the epilogue of their previous tile
-//    (tcgen05.ld of O in 16-column chunks, division by the row sum, 16-byte stores of the row).
+//    tcgen05.st of P, and the epilogue (tcgen05.ld of O, division by the row sum, 16-byte stores of
+//    the row), each warp taking whichever of its next softmax and its oldest epilogue is ready.
 //  * Every wait is bounded; on expiry the CTA records SD_ERR_TIMEOUT, drains and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -64,18 +64,15 @@ struct ShortCfg {
   static constexpr int V_OFF = K_OFF + KVB * K_BYTES;
   static constexpr int BAR_OFF = V_OFF + KVB * V_BYTES;
   // q_full[QS], q_empty[QS], k_full[KVB], v_full[KVB], v_ready[KVB], kv_empty[KVB], s_full[NSLOT],
-  // p_full[NSLOT], o_full[NSLOT], slot_free[NSLOT], fin
-  static constexpr int NBARS = 2 * QS + 4 * KVB + 4 * NSLOT + 1;
+  // p_full[NSLOT], o_full[NSLOT], slot_free[NSLOT], fin[2] (one per MMA-issuing warp)
+  static constexpr int NBARS = 2 * QS + 4 * KVB + 4 * NSLOT + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
-  // Warps: 0 TMA producer, 1 MMA issuer (and TMEM owner), 2 idle, 3 V fix-up; warpgroups 1 and 2
-  // run the softmax and epilogue of alternate tiles.
+  // Warps: 0 TMA producer, 1 S = Q K^T issuer (and TMEM owner), 2 O = P V issuer, 3 V fix-up;
+  // warpgroups 1 and 2 run the softmax and epilogue of alternate tiles.
   static constexpr int SOFT_WARP0 = 4;
   static constexpr int NWG = 2;
   static constexpr int THREADS = 128 + 128 * NWG;
-  // A warpgroup starts its next tile's softmax before its previous tile's epilogue when the two
-  // tiles sit in different slots and no other tile waits for that epilogue's slot in between.
-  static constexpr bool PIPE = NSLOT >= 3;
   static_assert(QS >= 1 && NSLOT >= 2, "resources");
   static_assert(NSLOT * TM_W <= 512, "tensor memory holds 512 columns");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -95,7 +92,7 @@ struct ShortBars {
   __device__ uint32_t p_full(int s) const { return base + 8 * (2 * C::QS + 4 * C::KVB + C::NSLOT + s); }
   __device__ uint32_t o_full(int s) const { return base + 8 * (2 * C::QS + 4 * C::KVB + 2 * C::NSLOT + s); }
   __device__ uint32_t slot_free(int s) const { return base + 8 * (2 * C::QS + 4 * C::KVB + 3 * C::NSLOT + s); }
-  __device__ uint32_t fin() const { return base + 8 * (2 * C::QS + 4 * C::KVB + 4 * C::NSLOT); }
+  __device__ uint32_t fin(int w) const { return base + 8 * (2 * C::QS + 4 * C::KVB + 4 * C::NSLOT + w); }
 };
 
 template <class C>
@@ -141,7 +138,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_init(bars.o_full(s), 1);
       mbar_init(bars.slot_free(s), 128);
     }
-    mbar_init(bars.fin(), 1);
+    mbar_init(bars.fin(0), 1);
+    mbar_init(bars.fin(1), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -206,82 +204,66 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         if (!(v_skipped && h == kv_issued - 1)) wait_bar(bars.v_full(h % KVB), (h / KVB) & 1, abort_flag, err, false);
       }
     } else if (warp == 1 && lane == 0) {
-      // ---------------------------------------------------------------- MMA issuer
-      // Two cursors over the tiles: S = Q K^T of tile iq (needs its Q, its head's K and a free
-      // slot) and O = P V of tile ip (needs its P and its head's V, with the ones column). P V goes
-      // first when both are ready.
+      // ---------------------------------------------------------------- S = Q K^T issuer
+      // Tiles in order: S of tile i needs its Q, its head's K and a free tensor-memory slot. The
+      // waits suspend the thread (no polling that would take issue slots from the softmax warps of
+      // this sub-partition); P V is issued by warp 2.
       constexpr uint32_t idesc_qk = idesc_f16kind_f32(BM, BN, false, C::F16);
-      constexpr uint32_t idesc_pv = idesc_f16kind_f32(BM, C::NPV, true, C::F16);
-      int iq = 0, ip = 0, hq = -1, hp = -1, prev_q = -1, prev_p = -1;
-      if (n > 0) {
-        hq = 0;
-        hp = 0;
-        prev_q = prev_p = head_of(0);
-      }
-      bool ok = true;
-      long long t_idle = clock64();
-      uint32_t spins = 0;
-      while (ok && ip < n) {
-        if (ip < iq) {
-          const int slot = ip % NSLOT, b = hp % KVB;
-          if (mbar_test_wait(bars.p_full(slot), (ip / NSLOT) & 1) &&
-              mbar_test_wait(bars.v_ready(b), (hp / KVB) & 1)) {
-            tc_fence_after();
-            const uint32_t d = tmem + slot * C::TM_W + BN, a = tmem + slot * C::TM_W;
+      int hq = 0, prev = n > 0 ? head_of(0) : -1;
+      for (int iq = 0; iq < n; ++iq) {
+        if (iq > 0 && head_of(iq) != prev) {
+          prev = head_of(iq);
+          ++hq;
+        }
+        const int slot = iq % NSLOT, qs = iq % QS, b = hq % KVB;
+        if (!wait_bar(bars.q_full(qs), (iq / QS) & 1, abort_flag, err) ||
+            !wait_bar(bars.k_full(b), (hq / KVB) & 1, abort_flag, err) ||
+            (iq >= NSLOT && !wait_bar(bars.slot_free(slot), (iq / NSLOT - 1) & 1, abort_flag, err)))
+          break;
+        tc_fence_after();
+        const uint32_t d = tmem + slot * C::TM_W;
 #pragma unroll
-            for (int ks = 0; ks < BN / 16; ++ks) {
-              const uint64_t bd = smem_desc(sbase + C::V_OFF + b * C::V_BYTES + ks * 16 * 128, BN * 128, 1024);
-              mma_ts(d, a + ks * 8, bd, idesc_pv, ks > 0 ? 1u : 0u);
-            }
-            mma_commit(bars.o_full(slot));
-            const bool last_of_head = ip + 1 == n || head_of(ip + 1) != prev_p;
-            if (last_of_head) mma_commit(bars.kv_empty(b));  // every P V of this head has been issued
-            ++ip;
-            if (ip < n && head_of(ip) != prev_p) {
-              prev_p = head_of(ip);
-              ++hp;
-            }
-            t_idle = clock64();
-            continue;
-          }
+        for (int ks = 0; ks < C::DHP / 16; ++ks) {
+          const uint32_t offq = (ks >> 2) * (BM * 128) + (ks & 3) * 32;
+          const uint32_t offk = (ks >> 2) * (BN * 128) + (ks & 3) * 32;
+          const uint64_t ad = smem_desc(sbase + C::Q_OFF + qs * C::Q_TILE + offq, 16, 1024);
+          const uint64_t bd = smem_desc(sbase + C::K_OFF + b * C::K_BYTES + offk, 16, 1024);
+          mma_ss(d, ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
         }
-        if (iq < n) {
-          const int slot = iq % NSLOT, qs = iq % QS, b = hq % KVB;
-          if (mbar_test_wait(bars.q_full(qs), (iq / QS) & 1) && mbar_test_wait(bars.k_full(b), (hq / KVB) & 1) &&
-              (iq < NSLOT || mbar_test_wait(bars.slot_free(slot), (iq / NSLOT - 1) & 1))) {
-            tc_fence_after();
-            const uint32_t d = tmem + slot * C::TM_W;
-#pragma unroll
-            for (int ks = 0; ks < C::DHP / 16; ++ks) {
-              const uint32_t offq = (ks >> 2) * (BM * 128) + (ks & 3) * 32;
-              const uint32_t offk = (ks >> 2) * (BN * 128) + (ks & 3) * 32;
-              const uint64_t ad = smem_desc(sbase + C::Q_OFF + qs * C::Q_TILE + offq, 16, 1024);
-              const uint64_t bd = smem_desc(sbase + C::K_OFF + b * C::K_BYTES + offk, 16, 1024);
-              mma_ss(d, ad, bd, idesc_qk, ks > 0 ? 1u : 0u);
-            }
-            mma_commit(bars.s_full(slot));
-            mma_commit(bars.q_empty(qs));
-            ++iq;
-            if (iq < n && head_of(iq) != prev_q) {
-              prev_q = head_of(iq);
-              ++hq;
-            }
-            t_idle = clock64();
-            continue;
-          }
-        }
-        if ((++spins & 31u) == 0) {
-          if (*abort_flag) ok = false;
-          else if (clock64() - t_idle > kWaitLimitCycles) {
-            *abort_flag = 1;
-            atomicOr(err, sd::kDevErrTimeout);
-            ok = false;
-          }
-        }
+        mma_commit(bars.s_full(slot));
+        mma_commit(bars.q_empty(qs));
       }
       // Drain: all tensor-core work issued by this thread completes before TMEM is released.
-      mma_commit(bars.fin());
-      wait_bar(bars.fin(), 0, abort_flag, err, false);
+      mma_commit(bars.fin(0));
+      wait_bar(bars.fin(0), 0, abort_flag, err, false);
+    } else if (warp == 2 && lane == 0) {
+      // ---------------------------------------------------------------- O = P V issuer
+      // Tiles in order: P V of tile i needs its P (written over S by the softmax) and its head's V
+      // with the ones column. After the last P V of a head the K/V buffer is released: every S of
+      // that head has completed, since each P V waited for its tile's softmax.
+      constexpr uint32_t idesc_pv = idesc_f16kind_f32(BM, C::NPV, true, C::F16);
+      int hp = 0, prev = n > 0 ? head_of(0) : -1;
+      for (int ip = 0; ip < n; ++ip) {
+        if (ip > 0 && head_of(ip) != prev) {
+          prev = head_of(ip);
+          ++hp;
+        }
+        const int slot = ip % NSLOT, b = hp % KVB;
+        if (!wait_bar(bars.p_full(slot), (ip / NSLOT) & 1, abort_flag, err) ||
+            !wait_bar(bars.v_ready(b), (hp / KVB) & 1, abort_flag, err))
+          break;
+        tc_fence_after();
+        const uint32_t d = tmem + slot * C::TM_W + BN, a = tmem + slot * C::TM_W;
+#pragma unroll
+        for (int ks = 0; ks < BN / 16; ++ks) {
+          const uint64_t bd = smem_desc(sbase + C::V_OFF + b * C::V_BYTES + ks * 16 * 128, BN * 128, 1024);
+          mma_ts(d, a + ks * 8, bd, idesc_pv, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(bars.o_full(slot));
+        if (ip + 1 == n || head_of(ip + 1) != prev) mma_commit(bars.kv_empty(b));
+      }
+      mma_commit(bars.fin(1));
+      wait_bar(bars.fin(1), 0, abort_flag, err, false);
     } else if (warp == 3) {
       // ---------------------------------------------------------------- V fix-up
       // Writes 1.0 into column DH of every row of each landed V buffer (128-byte swizzled rows: the
@@ -425,14 +407,34 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       return true;
     };
 
-    if constexpr (C::PIPE) {
-      for (int i = wg; ok && i < n + C::NWG; i += C::NWG) {
-        if (i < n && !softmax(i)) ok = false;
-        if (ok && i - C::NWG >= 0 && i - C::NWG < n && !epilogue(i - C::NWG)) ok = false;
+    // Each warp takes whichever of its warpgroup's next steps is ready: the epilogue of its oldest
+    // tile whose O is complete, else the softmax of its next tile whose S is complete. Probing a
+    // barrier of tile i only after this warp finished tile i - NWG is safe: the issuers work in tile
+    // order and a commit covers all of the issuing thread's earlier MMAs, so the slot's previous phase
+    // has completed and a parity probe cannot see a stale phase.
+    int ns = wg, ne = wg;  // next tile to softmax, next tile to write out
+    long long t_idle = clock64();
+    uint32_t spins = 0;
+    while (ok && ne < n) {
+      if (ne < ns && __all_sync(0xffffffffu, mbar_test_wait(bars.o_full(ne % NSLOT), (ne / NSLOT) & 1))) {
+        if (!epilogue(ne)) ok = false;
+        ne += C::NWG;
+        t_idle = clock64();
+        continue;
       }
-    } else {
-      for (int i = wg; ok && i < n; i += C::NWG) {
-        if (!softmax(i) || !epilogue(i)) ok = false;
+      if (ns < n && __all_sync(0xffffffffu, mbar_test_wait(bars.s_full(ns % NSLOT), (ns / NSLOT) & 1))) {
+        if (!softmax(ns)) ok = false;
+        ns += C::NWG;
+        t_idle = clock64();
+        continue;
+      }
+      if ((++spins & 31u) == 0) {
+        if (*abort_flag) ok = false;
+        else if (clock64() - t_idle > kWaitLimitCycles) {
+          *abort_flag = 1;
+          atomicOr(err, sd::kDevErrTimeout);
+          ok = false;
+        }
       }
     }
   }
