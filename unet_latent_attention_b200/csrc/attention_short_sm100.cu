@@ -33,6 +33,9 @@
 #ifndef SD_SHORT_POLY
 #define SD_SHORT_POLY 2
 #endif
+#ifndef SD_SHORT_PERSIST
+#define SD_SHORT_PERSIST 0  // 1: the persistent multi-tile form instead of one query tile per CTA
+#endif
 
 namespace {
 
@@ -488,9 +491,291 @@ sd_status launch_cfg(const void* q, const void* k, const void* v, void* o, int64
                         "sd_attention (short key sequence) launch");
 }
 
+// ------------------------------------------------------------------ one query tile per CTA
+// The default form: a CTA takes one 128-row query tile, so the GPU runs several tiles' chains
+// (loads, S, softmax, P V, stores) at once on every SM and their latencies overlap; three to four
+// of these CTAs fit one SM. Tensor memory of a CTA: S in columns [0, 80), P written over its first
+// 40 columns, and O (then the row sum for L_IN_V) from column OFS_O, over the columns of S that the
+// softmax has already read: 128 columns for dh 40 and 64, 256 for dh 80 and 160.
+template <int DH_, bool F16_, bool BLHD_>
+struct TileCfg {
+  static constexpr int DH = DH_;
+  static constexpr bool F16 = F16_;
+  static constexpr bool BLHD = BLHD_;
+  static constexpr int BN = kShortMaxKeys;
+  static constexpr int POLY = SD_SHORT_POLY;
+  static constexpr int DHP = (DH + 15) / 16 * 16;
+  static constexpr bool L_IN_V = DH != 64;  // the row sum from a ones column, except where it would widen V
+  static constexpr int NPV = L_IN_V ? (DH + 1 + 15) / 16 * 16 : DHP;
+  static constexpr int NCH = (DHP + 63) / 64;
+  static constexpr int NCHV = (NPV + 63) / 64;
+  static constexpr int Q_BYTES = NCH * BM * 128;
+  static constexpr int K_BYTES = NCH * BN * 128;
+  static constexpr int V_BYTES = NCHV * BN * 128;
+  static constexpr int Q_OFF = 0, K_OFF = Q_BYTES, V_OFF = K_OFF + K_BYTES;
+  static constexpr int BAR_OFF = V_OFF + V_BYTES;
+  // qk_full, v_full, v_ready, s_full, p_full, o_full, fin
+  static constexpr int NBARS = 7;
+  static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static constexpr int OFS_O = BN / 2 + 8;  // past P (BN / 2 columns), 16-aligned
+  static constexpr int TM_COLS = OFS_O + NPV <= 128 ? 128 : 256;
+  static constexpr int THREADS = 160;  // warp 0: loads, MMAs, V fix-up; warps 1-4: softmax, epilogue
+  static_assert(OFS_O % 16 == 0 && OFS_O + NPV <= TM_COLS, "tensor-memory layout");
+};
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS)
+    attn_tile_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out, int Lq, int Lk, int dh,
+                    float scale_log2, unsigned int* err, int debug_flags, int tiles_per_head, int lay_heads) {
+  constexpr int BN = C::BN, NCH = C::NCH, NCHV = C::NCHV;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar = sbase + C::BAR_OFF;
+  const uint32_t qk_full = bar, v_full = bar + 8, v_ready = bar + 16, s_full = bar + 24, p_full = bar + 32,
+                 o_full = bar + 40, fin = bar + 48;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = static_cast<int>(blockIdx.x / static_cast<unsigned>(tiles_per_head));
+  const int row0 = static_cast<int>(blockIdx.x % static_cast<unsigned>(tiles_per_head)) * BM;
+
+  if (threadIdx.x == 0) {
+    mbar_init(qk_full, 1);
+    mbar_init(v_full, 1);
+    mbar_init(v_ready, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(o_full, 1);
+    mbar_init(fin, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), C::TM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  sd::grid_dep_wait();
+  sd::grid_dep_launch();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // loads, then S = Q K^T once Q and K have landed, then O = P V once P is written
+      mbar_arrive_expect_tx(qk_full, C::Q_BYTES + C::K_BYTES);
+      for (int c = 0; c < NCH; ++c) {
+        load_rows<C::BLHD>(sbase + C::Q_OFF + c * BM * 128, &tm_q, qk_full, c * 64, row0, bh, lay_heads);
+        load_rows<C::BLHD>(sbase + C::K_OFF + c * BN * 128, &tm_k, qk_full, c * 64, 0, bh, lay_heads);
+      }
+      const bool skip_v = debug_flags & 1;  // test hook: V never arrives, the waits below expire
+      if (!skip_v) {
+        mbar_arrive_expect_tx(v_full, C::V_BYTES);
+        for (int c = 0; c < NCHV; ++c)
+          load_rows<C::BLHD>(sbase + C::V_OFF + c * BN * 128, &tm_v, v_full, c * 64, 0, bh, lay_heads);
+      }
+      constexpr uint32_t idesc_qk = idesc_f16kind_f32(BM, BN, false, C::F16);
+      constexpr uint32_t idesc_pv = idesc_f16kind_f32(BM, C::NPV, true, C::F16);
+      bool issued_pv = false;
+      if (wait_bar(qk_full, 0, abort_flag, err)) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < C::DHP / 16; ++ks) {
+          const uint32_t off = (ks >> 2) * (BM * 128) + (ks & 3) * 32;
+          const uint32_t offk = (ks >> 2) * (BN * 128) + (ks & 3) * 32;
+          mma_ss(tmem, smem_desc(sbase + C::Q_OFF + off, 16, 1024), smem_desc(sbase + C::K_OFF + offk, 16, 1024),
+                 idesc_qk, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full);
+        if (wait_bar(p_full, 0, abort_flag, err) && wait_bar(C::L_IN_V ? v_ready : v_full, 0, abort_flag, err)) {
+          tc_fence_after();
+#pragma unroll
+          for (int ks = 0; ks < BN / 16; ++ks)
+            mma_ts(tmem + C::OFS_O, tmem + ks * 8, smem_desc(sbase + C::V_OFF + ks * 16 * 128, BN * 128, 1024), idesc_pv,
+                   ks > 0 ? 1u : 0u);
+          mma_commit(o_full);
+          issued_pv = true;
+        }
+      }
+      mma_commit(fin);
+      wait_bar(fin, 0, abort_flag, err, false);
+      // drain: the copies issued above have landed before the CTA may exit
+      wait_bar(qk_full, 0, abort_flag, err, false);
+      if (!skip_v) wait_bar(v_full, 0, abort_flag, err, false);
+      (void)issued_pv;
+    } else if constexpr (C::L_IN_V) {
+      // V fix-up: 1.0 in column DH of every key row (128-byte swizzle: granule g of row r at g ^ (r % 8))
+      constexpr int ch = C::DH / 64, byte = (C::DH % 64) * 2, g = byte >> 4, gb = byte & 15;
+      if (__all_sync(0xfffffffeu, wait_bar(v_full, 0, abort_flag, err))) {
+        uint8_t* vt = smem + C::V_OFF + ch * BN * 128;
+        for (int r = lane - 1; r < BN; r += 31)
+          *reinterpret_cast<uint16_t*>(vt + r * 128 + ((g ^ (r & 7)) << 4) + gb) = C::F16 ? 0x3C00u : 0x3F80u;
+        fence_proxy_async_smem();
+        __syncwarp(0xfffffffeu);
+        if (lane == 1) mbar_arrive(v_ready);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- softmax and epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    if (__all_sync(0xffffffffu, wait_bar(s_full, 0, abort_flag, err))) {
+      tc_fence_after();
+      float sv[BN];
+      {
+        uint32_t r0[32], r1[32], r2[16];
+        tmem_ld32(tl, r0);
+        tmem_ld32(tl + 32, r1);
+        tmem_ld16(tl + 64, r2);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sv[j] = __uint_as_float(r0[j]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) sv[32 + j] = __uint_as_float(r1[j]);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) sv[64 + j] = __uint_as_float(r2[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < BN; ++j)
+        if (j >= Lk) sv[j] = -INFINITY;
+      float pm[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) pm[k] = max3f(sv[k], sv[16 + k], sv[32 + k]);
+#pragma unroll
+      for (int k = 0; k < 16; ++k) pm[k] = max3f(pm[k], sv[48 + k], sv[64 + k]);
+      const float mx = fmaxf(max3f(max3f(pm[0], pm[1], pm[2]), max3f(pm[3], pm[4], pm[5]), max3f(pm[6], pm[7], pm[8])),
+                             max3f(max3f(pm[9], pm[10], pm[11]), max3f(pm[12], pm[13], pm[14]), pm[15]));
+      const float neg_m = -mx * scale_log2;
+      uint32_t pk[BN / 2];
+      float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+      for (int b = 0; b < BN / 2; ++b) {
+        float x0, x1;
+        fma2(x0, x1, sv[2 * b], sv[2 * b + 1], scale_log2, scale_log2, neg_m, neg_m);
+        if ((b & 7) < C::POLY) {
+          exp2_poly2(x0, x1, x0, x1);
+        } else {
+          x0 = ex2_approx(x0);
+          x1 = ex2_approx(x1);
+        }
+        if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x0, x1);
+        pk[b] = C::F16 ? pack_f16x2(x0, x1) : pack_bf16x2(x0, x1);
+      }
+      {
+        uint32_t a[16], c[16], e[8];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) a[j] = pk[j];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) c[j] = pk[16 + j];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) e[j] = pk[32 + j];
+        tmem_st16(tl, a);
+        tmem_st16(tl + 16, c);
+        tmem_st8(tl + 32, e);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full);
+      if (__all_sync(0xffffffffu, wait_bar(o_full, 0, abort_flag, err))) {
+        tc_fence_after();
+        const uint32_t tO = tl + C::OFS_O;
+        const int qrow = row0 + row;
+        const size_t orow = C::BLHD ? (static_cast<size_t>(bh / lay_heads) * Lq + qrow) * lay_heads + bh % lay_heads
+                                    : static_cast<size_t>(bh) * Lq + qrow;
+        uint4* dst = reinterpret_cast<uint4*>(out + orow * dh);
+        float inv_l;
+        if constexpr (C::L_IN_V) {
+          uint32_t lc[16];
+          tmem_ld16(tO + (C::DH / 16) * 16, lc);
+          tmem_wait_ld();
+          inv_l = 1.0f / __uint_as_float(lc[C::DH % 16]);
+        } else {
+          inv_l = 1.0f / (ls0 + ls1);
+        }
+#pragma unroll 2
+        for (int c = 0; c < C::DH / 16 + (C::DH % 16 ? 1 : 0); ++c) {
+          uint32_t r[16];
+          tmem_ld16(tO + c * 16, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (c * 2 + h >= C::DH / 8) break;
+            uint32_t w[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              w[j] = C::F16 ? pack_f16x2(__uint_as_float(r[8 * h + 2 * j]) * inv_l, __uint_as_float(r[8 * h + 2 * j + 1]) * inv_l)
+                            : pack_bf16x2(__uint_as_float(r[8 * h + 2 * j]) * inv_l, __uint_as_float(r[8 * h + 2 * j + 1]) * inv_l);
+            if (qrow < Lq) dst[c * 2 + h] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TM_COLS);
+  }
+}
+
+template <class C>
+sd_status launch_tile(const void* q, const void* k, const void* v, void* o, int64_t BH, int64_t Lq, int64_t Lk,
+                      int64_t dh, float scale, cudaStream_t s, int64_t lay_heads) {
+  CUtensorMap mq, mk, mv;
+  sd_status st = make_map(&mq, q, dh, Lq, BH, BM, C::F16, lay_heads);
+  if (st == SD_OK) st = make_map(&mk, k, dh, Lk, BH, C::BN, C::F16, lay_heads);
+  if (st == SD_OK) st = make_map(&mv, v, dh, Lk, BH, C::BN, C::F16, lay_heads);
+  if (st != SD_OK) return st;
+  unsigned int* err = sd::device_status_word();
+  if (!err) return SD_ERR_CUDA;
+  auto kern = attn_tile_sm100<C>;
+  static std::atomic<uint64_t> smem_set{0};
+  int dev = 0;
+  st = sd::cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st != SD_OK) return st;
+  const uint64_t bit = uint64_t(1) << (dev & 63);
+  if (!(smem_set.load(std::memory_order_acquire) & bit)) {
+    st = sd::cuda_check(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES),
+                        "cudaFuncSetAttribute(tile attention smem)");
+    if (st != SD_OK) return st;
+    smem_set.fetch_or(bit, std::memory_order_acq_rel);
+  }
+  const int64_t tph = (Lq + BM - 1) / BM;
+  const int64_t n_tiles = BH * tph;
+  if (n_tiles > 0x7fffffff) return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention: too many query tiles");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(n_tiles));
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  cfg.attrs = attr;
+  cfg.numAttrs = sd::pdl_attr(&attr[0]);
+  return sd::cuda_check(cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, static_cast<uint16_t*>(o), static_cast<int>(Lq),
+                                           static_cast<int>(Lk), static_cast<int>(dh), scale * 1.4426950408889634f, err,
+                                           g_debug_flags, static_cast<int>(tph), static_cast<int>(lay_heads)),
+                        "sd_attention (one query tile per CTA) launch");
+}
+
 template <bool F16, bool BLHD>
 sd_status dispatch_dh(const void* q, const void* k, const void* v, void* o, int64_t BH, int64_t Lq, int64_t Lk,
                       int64_t dh, float scale, cudaStream_t s, int64_t lay_heads) {
+  if (!SD_SHORT_PERSIST) {
+    switch (dh) {
+      case 40: return launch_tile<TileCfg<40, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, lay_heads);
+      case 64: return launch_tile<TileCfg<64, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, lay_heads);
+      case 80: return launch_tile<TileCfg<80, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, lay_heads);
+      case 160: return launch_tile<TileCfg<160, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, lay_heads);
+      default: return sd::fail(SD_ERR_UNSUPPORTED, "sd_attention: head dim %lld", (long long)dh);
+    }
+  }
   switch (dh) {
     case 40: return launch_cfg<ShortCfg<40, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, lay_heads);
     case 64: return launch_cfg<ShortCfg<64, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, lay_heads);
