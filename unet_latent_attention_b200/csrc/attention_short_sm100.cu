@@ -34,7 +34,7 @@
 #define SD_SHORT_POLY 2
 #endif
 #ifndef SD_SHORT_PERSIST
-#define SD_SHORT_PERSIST 0  // 1: the persistent multi-tile form instead of one query tile per CTA
+#define SD_SHORT_PERSIST 0  // 1: always the persistent multi-tile form (never one query tile per CTA)
 #endif
 
 namespace {
@@ -525,7 +525,7 @@ struct TileCfg {
 };
 
 template <class C>
-__global__ void __launch_bounds__(C::THREADS)
+__global__ void __launch_bounds__(C::THREADS, C::TM_COLS == 128 ? 4 : 2)
     attn_tile_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, uint16_t* __restrict__ out, int Lq, int Lk, int dh,
                     float scale_log2, unsigned int* err, int debug_flags, int tiles_per_head, int lay_heads) {
@@ -767,7 +767,11 @@ sd_status launch_tile(const void* q, const void* k, const void* v, void* o, int6
 template <bool F16, bool BLHD>
 sd_status dispatch_dh(const void* q, const void* k, const void* v, void* o, int64_t BH, int64_t Lq, int64_t Lk,
                       int64_t dh, float scale, cudaStream_t s, int64_t lay_heads) {
-  if (!SD_SHORT_PERSIST) {
+  // One tile per CTA while every tile fits one wave of resident CTAs (their chains then overlap);
+  // beyond that, the persistent form, whose CTAs keep up to 8 tiles' loads in flight.
+  const int64_t n_tiles = BH * ((Lq + BM - 1) / BM);
+  const int per_sm = (dh == 40 || dh == 64) ? 4 : 2;  // the tile kernel's resident CTAs per SM
+  if (!SD_SHORT_PERSIST && n_tiles <= static_cast<int64_t>(per_sm) * sd::sm_count()) {
     switch (dh) {
       case 40: return launch_tile<TileCfg<40, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, lay_heads);
       case 64: return launch_tile<TileCfg<64, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, lay_heads);
