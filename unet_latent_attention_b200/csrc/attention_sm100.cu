@@ -110,10 +110,6 @@ enum : int { kSplitPublish = 1, kSplitMerge = 2, kSplitAbort = 3 };  // split ha
 #define SD_PING_RELEASE -1  // tuning override of Cfg::PING_RELEASE (-1: the per-config choice)
 #endif
 
-#ifndef SD_NQ3
-#define SD_NQ3 0  // three query tiles per CTA for long query sequences (dh 40 and 64)
-#endif
-
 #ifndef SD_REGSPLIT
 #define SD_REGSPLIT 0  // setmaxnreg: 56 registers per helper thread, 224 per softmax thread
 #endif
@@ -179,41 +175,31 @@ struct Cfg {
   static constexpr int V_OFF = K_OFF + STAGES * K_TILE_BYTES;
   static constexpr int BAR_OFF = V_OFF + STAGES * V_TILE_BYTES;
   // q_full, k_full[S], v_full[S], v_ready[S], kv_empty[S], s_full[NQ], s_free[NQ], p_full[NQ], o_done[NQ],
-  // fin[NQ], the exp tokens tok[NQ][4] of the tiles' warps on each SM sub-partition, q_empty[2],
+  // fin[NQ], the exp tokens tok[2][4] of the two tiles' warps on each SM sub-partition, q_empty[2],
   // split_dec[2], split_written[2]
-  static constexpr int NBARS = 2 + 4 * STAGES + 9 * NQ + 2 + 4;
+  static constexpr int NBARS = 2 + 4 * STAGES + 5 * NQ + 8 + 2 + 4;
   static constexpr int MISC_OFF = BAR_OFF + NBARS * 8;
   // misc: TMEM base address, abort flag, the split hand-off decisions of the two piece kinds
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
-  // TMEM columns. NQ <= 2: one 256- or 512-column block per query tile, S | P (if separate) | O
-  // (NPV columns, l at column DH). NQ = 3 (three tiles in 512 columns): the three S blocks, then the
-  // three O blocks, then the three P blocks, each start a multiple of 16 (S, O) or 8 (P) columns.
+  // TMEM columns of one query tile: S | P (if separate) | O (NPV columns, l at column DH)
   static constexpr int TM_S = 0;
   static constexpr int TM_P = P_SEP ? BN : 0;
   static constexpr int TM_O = BN + (P_SEP ? BN / 2 : 0);
   static constexpr int TM_USED = TM_O + NPV;
   static constexpr int TM_TILE = TM_USED <= 256 ? 256 : 512;
-  static constexpr int TM_COLS = NQ == 3 ? 512 : NQ * TM_TILE;
-  static constexpr __host__ __device__ int s_col(int t) { return NQ == 3 ? t * BN : t * TM_TILE + TM_S; }
-  static constexpr __host__ __device__ int o_col(int t) { return NQ == 3 ? 3 * BN + t * NPV : t * TM_TILE + TM_O; }
-  static constexpr __host__ __device__ int p_col(int t) {
-    return NQ == 3 ? (P_SEP ? 3 * BN + 3 * NPV + t * (BN / 2) : t * BN) : t * TM_TILE + TM_P;
-  }
-  // Warpgroup 0 holds the helpers -- warp 0: TMA producer (lane 0; with three tiles lanes 1-31 do
-  // the V fix-up); warps 1 .. NQ: the MMA issuer of one query tile each (warp 1 owns TMEM); warp 3
-  // (up to two tiles): V fix-up (L_IN_V) -- and warpgroups 1 .. NQ run the softmax of one query tile
-  // each (warp w reads TMEM lane quarter w % 4).
-  static_assert(NQ <= 3, "three MMA issuers in warpgroup 0");
-  static constexpr int FIX_WARP = NQ == 3 ? 0 : 3;
+  static constexpr int TM_COLS = NQ * TM_TILE;
+  // Warpgroup 0 holds the helpers -- warp 0: TMA producer; warp 1: MMA issuer of tile 0 (and TMEM
+  // owner); warp 2: MMA issuer of tile 1; warp 3: V fix-up (L_IN_V) -- and warpgroups 1 .. NQ run
+  // the softmax of one query tile each (warp w reads TMEM lane quarter w % 4).
+  static_assert(NQ <= 2, "two MMA issuers in warpgroup 0");
+  static constexpr int FIX_WARP = 3;
   static constexpr int SOFT_WARP0 = 4;
   static constexpr int NUM_WARPS = 4 + 4 * NQ;
   static constexpr int THREADS = 32 * NUM_WARPS;
-  // Register split (setmaxnreg): the helper warpgroup drops to REG_HELPER per thread and the softmax
-  // warpgroups rise to REG_SOFT. Optional for NQ = 2 (384 x 168 at launch); always for NQ = 3, whose
-  // 512 threads launch with 128 each.
-  static constexpr int REG_HELPER = NQ == 3 ? 48 : 56, REG_SOFT = NQ == 3 ? 152 : 224;
-  static constexpr bool REG_SPLIT = NQ == 3 || (SD_REGSPLIT && NQ == 2);
-  static_assert(!REG_SPLIT || 128 * REG_HELPER + 128 * NQ * REG_SOFT <= 65536, "register split exceeds the launch budget");
+  // Register split (setmaxnreg) for NQ = 2: the helper warpgroup drops to REG_HELPER per thread and
+  // the two softmax warpgroups rise to REG_SOFT, within the launch's 384 x 168.
+  static constexpr int REG_HELPER = 56, REG_SOFT = 224;
+  static_assert(NQ != 2 || 128 * REG_HELPER + 256 * REG_SOFT <= 168 * 384, "register split exceeds the launch budget");
   // Split-item hand-off slot: raw O (NPV fp32 per row) and (m, l) per row of the NQ tiles.
   static constexpr int SLOT_FLOATS = NQ * BM * (NPV + 2);
   // Column pairs after which a softmax warp passes the ping-pong token (measured: half-way for
@@ -221,16 +207,15 @@ struct Cfg {
   static constexpr int PING_RELEASE = (DH == 64 && BN == 128) ? BN / 4 : BN / 2;
   // Store P in 16-column chunks inside the exp2 loop (measured: faster for the single short key
   // tile of cross-attention, slower for the long key loops).
-  static constexpr bool CHUNK_P = BN < 128 && NQ <= 2;
+  static constexpr bool CHUNK_P = BN < 128;
   // Costs of the persistent schedule in K/V-tile units (measured; see part_ranges).
   static constexpr double COST_SEG = DH == 64 ? 1.3 : 1.0, COST_TAIL = DH == 64 ? 0.5 : 0.6,
                           COST_HEAD = DH == 64 ? 1.4 : 0.9;
   // Of every 8 column pairs, this many take the FMA-pipe exp2 instead of the special-function unit.
   static constexpr int POLY_PAIRS = SD_POLY_PAIRS >= 0 ? SD_POLY_PAIRS : POLY_;
   static_assert(NPV % 16 == 0 && NPV <= 256, "MMA N must be a multiple of 16 and at most 256");
-  static_assert(BN % 16 == 0, "S is read in 32-column chunks and a 16-column tail");
+  static_assert(BN % 32 == 0, "S is read in 32-column chunks");
   static_assert(TM_COLS <= 512, "tensor memory holds 512 columns");
-  static_assert(NQ != 3 || 3 * (BN + NPV) + (P_SEP ? 3 * (BN / 2) : 0) <= 512, "three tiles in tensor memory");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 };
 
@@ -248,11 +233,11 @@ struct Bars {
   __device__ uint32_t o_done(int t) const { return base + 8 * (2 + 4 * stages + 3 * nq + t); }
   __device__ uint32_t fin() const { return base + 8 * (2 + 4 * stages + 4 * nq); }
   __device__ uint32_t tok(int t, int q) const { return base + 8 * (2 + 4 * stages + 5 * nq + 4 * t + q); }
-  __device__ uint32_t q_empty(int b) const { return base + 8 * (2 + 4 * stages + 9 * nq + b); }
+  __device__ uint32_t q_empty(int b) const { return base + 8 * (2 + 4 * stages + 5 * nq + 8 + b); }
   // split-item hand-off of the tail piece (kind 0) and the head piece (kind 1): the leader's
   // decision is published, and this piece's slot has been written by every softmax thread
-  __device__ uint32_t split_dec(int kind) const { return base + 8 * (2 + 4 * stages + 9 * nq + 2 + kind); }
-  __device__ uint32_t split_written(int kind) const { return base + 8 * (2 + 4 * stages + 9 * nq + 4 + kind); }
+  __device__ uint32_t split_dec(int kind) const { return base + 8 * (2 + 4 * stages + 5 * nq + 10 + kind); }
+  __device__ uint32_t split_written(int kind) const { return base + 8 * (2 + 4 * stages + 5 * nq + 12 + kind); }
 };
 
 // Persistent schedule: the work is items x nkv units (an item = NQ query tiles of one (b, h); a
@@ -320,7 +305,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_init(bars.o_done(t), 1);
     }
     for (int t = 0; t < NQ; ++t) mbar_init(bars.fin() + 8 * t, 1);
-    for (int i = 0; i < 4 * NQ; ++i) mbar_init(bars.tok(i >> 2, i & 3), 1);
+    for (int i = 0; i < 8; ++i) mbar_init(bars.tok(i >> 2, i & 3), 1);
     mbar_init(bars.q_empty(0), NQ);
     mbar_init(bars.q_empty(1), NQ);
     for (int kind = 0; kind < 2; ++kind) {
@@ -348,28 +333,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   sd::grid_dep_wait();
   sd::grid_dep_launch();
 
-  // V fix-up: writes 1.0 (bf16 or fp16) into column DH of every landed V tile (128-byte swizzled
-  // rows: the 16-byte granule g of row r sits at granule g ^ (r % 8)), then hands the tile to the MMA
-  // issuers, so that P V also sums each row of P. Run by the lanes in `mask` (first lane `lead`,
-  // `nl` lanes): all of warp 3, or lanes 1-31 of warp 0 beside the TMA producer on lane 0.
-  auto fix_v = [&](unsigned mask, int lead, int nl) {
-    constexpr int ch = C::DH / 64, byte = (C::DH % 64) * 2, g = byte >> 4, gb = byte & 15;
-    const int total = static_cast<int>(u1 - u0);  // K/V tiles this CTA streams
-    for (int j = 0; j < total; ++j) {
-      const int s = j % STAGES;
-      if (!__all_sync(mask, wait_bar(bars.v_full(s), (j / STAGES) & 1, abort_flag, err))) break;
-      uint8_t* vt = smem + C::V_OFF + s * C::V_TILE_BYTES + ch * BN * 128;
-      for (int r = lane - lead; r < BN; r += nl)
-        *reinterpret_cast<uint16_t*>(vt + r * 128 + ((g ^ (r & 7)) << 4) + gb) = C::F16 ? 0x3C00u : 0x3F80u;  // 1.0
-      fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
-      __syncwarp(mask);
-      if (lane == lead) mbar_arrive(bars.v_ready(s));
-    }
-  };
-
   if (warp < C::SOFT_WARP0) {
   // ==================================================================== helper warpgroup
-  if constexpr (C::REG_SPLIT) regs_dec<C::REG_HELPER>();  // registers move to the softmax warpgroups
+  if constexpr (SD_REGSPLIT && NQ == 2) regs_dec<C::REG_HELPER>();  // registers move to the softmax warpgroups
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -422,11 +388,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           if (!((debug_flags & 1) && s == 0 && issued[s] == 1))
             wait_bar(bars.v_full(s), (issued[s] - 1) & 1, abort_flag, err, false);
         }
-    } else if constexpr (C::L_IN_V && C::FIX_WARP == 0) {
-      fix_v(0xfffffffeu, 1, 31);
     }
-    __syncwarp();
-  } else if (warp >= 1 && warp <= NQ) {
+  } else if (warp == 1 || (NQ == 2 && warp == 2)) {
     // ------------------------------------------------------------------ MMA issuer of one tile
     // One issuing warp per query tile: a tcgen05.mma occupies its issuing thread for tens to
     // hundreds of cycles, so two tiles' instruction streams must not queue behind each other.
@@ -436,7 +399,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       constexpr uint32_t idesc_pv = idesc_f16kind_f32(BM, C::NPV, true, C::F16);
       uint32_t tq = sbase + C::Q_OFF + t * C::Q_TILE_BYTES;  // the current segment's Q buffer
       auto issue_qk = [&](int s) {  // S = Q K_s^T over the padded head dim
-        const uint32_t d = tmem + C::s_col(t);
+        const uint32_t d = tmem + t * C::TM_TILE + C::TM_S;
 #pragma unroll
         for (int ks = 0; ks < DHP / 16; ++ks) {
           const uint32_t off = (ks >> 2) * (BM * 128) + (ks & 3) * 32;
@@ -447,8 +410,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
       };
       auto issue_pv = [&](int s, bool first) {  // O (+)= P V_s, P from TMEM (16 keys = 8 columns)
-        const uint32_t d = tmem + C::o_col(t);
-        const uint32_t a = tmem + C::p_col(t);
+        const uint32_t d = tmem + t * C::TM_TILE + C::TM_O;
+        const uint32_t a = tmem + t * C::TM_TILE + C::TM_P;
 #pragma unroll
         for (int ks = 0; ks < BN / 16; ++ks) {
           const uint64_t b = smem_desc(sbase + C::V_OFF + s * C::V_TILE_BYTES + ks * 16 * 128, BN * 128, 1024);
@@ -568,7 +531,23 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     __syncwarp();
   } else if (C::L_IN_V && warp == C::FIX_WARP) {
-    fix_v(0xffffffffu, 0, 32);
+
+    // ------------------------------------------------------------------ V fix-up warp
+    // Writes bf16 1.0 into column DH of every landed V tile (128-byte swizzled rows: the 16-byte
+    // granule g of row r sits at granule g ^ (r % 8)), then hands the tile to the MMA issuer.
+    constexpr int ch = C::DH / 64, byte = (C::DH % 64) * 2, g = byte >> 4, gb = byte & 15;
+    const int total = static_cast<int>(u1 - u0);  // K/V tiles this CTA streams
+    for (int j = 0; j < total; ++j) {
+      const int s = j % STAGES;
+      if (!__all_sync(0xffffffffu, wait_bar(bars.v_full(s), (j / STAGES) & 1, abort_flag, err))) break;
+      uint8_t* vt = smem + C::V_OFF + s * C::V_TILE_BYTES + ch * BN * 128;
+#pragma unroll
+      for (int r = lane; r < BN; r += 32)
+        *reinterpret_cast<uint16_t*>(vt + r * 128 + ((g ^ (r & 7)) << 4) + gb) = C::F16 ? 0x3C00u : 0x3F80u;  // 1.0
+      fence_proxy_async_smem();  // generic-proxy stores -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.v_ready(s));
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -578,16 +557,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   }
   } else {
   // ==================================================================== softmax warpgroups
-  if constexpr (C::REG_SPLIT) regs_inc<C::REG_SOFT>();
+  if constexpr (SD_REGSPLIT && NQ == 2) regs_inc<C::REG_SOFT>();
   {
     // ------------------------------------------------------------------ softmax warps
     const int t = (warp - C::SOFT_WARP0) >> 2;  // query tile of this warpgroup
     const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
-    const uint32_t tbase = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    const uint32_t tS = tbase + C::s_col(t), tP = tbase + C::p_col(t), tO = tbase + C::o_col(t);
+    const uint32_t tbase = tmem + t * C::TM_TILE + (static_cast<uint32_t>(quarter * 32) << 16);
+    const uint32_t tS = tbase + C::TM_S, tP = tbase + C::TM_P, tO = tbase + C::TM_O;
     bool ok = true;
-    constexpr bool kPing = SD_PINGPONG && NQ >= 2 && (SD_PING_SHORT || BN == 128);
+    constexpr bool kPing = SD_PINGPONG && NQ == 2 && (SD_PING_SHORT || BN == 128);
     long long u = u0;
     Seg sg;
     int gi = 0;  // CTA-wide K/V tile count: the phase of every per-tile barrier
@@ -610,12 +589,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tmem_ld32(tS + c * 32, r);
 #pragma unroll
         for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(r[i]);
-      }
-      if constexpr (BN % 32 == 16) {
-        uint32_t r[16];
-        tmem_ld16(tS + BN - 16, r);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) sv[BN - 16 + i] = __uint_as_float(r[i]);
       }
       tmem_wait_ld();
       if constexpr (C::P_SEP) {  // S is in registers: the next S = Q K^T may overwrite it
@@ -676,8 +649,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // Ping-pong: the special-function unit of a sub-partition serves one tile's exp2 phase at a
       // time; the other tile's warp on it does its row max, P store and S load meanwhile. Tile 0
       // goes first; each warp hands the token to its partner (same sub-partition) after its exps.
-      if (kPing && (t > 0 || gi > 0)) {
-        if (!__all_sync(0xffffffffu, wait_bar(bars.tok(t, quarter), (t > 0 ? gi : gi - 1) & 1, abort_flag, err))) {
+      if (kPing && (t == 1 || gi > 0)) {
+        if (!__all_sync(0xffffffffu, wait_bar(bars.tok(t, quarter), (t == 1 ? gi : gi - 1) & 1, abort_flag, err))) {
           ok = false;
           break;
         }
@@ -709,7 +682,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           pk[b] = C::F16 ? pack_f16x2(x0, x1) : pack_bf16x2(x0, x1);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(bars.tok(t + 1 == NQ ? 0 : t + 1, quarter));
+        if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
 #pragma unroll
         for (int b = 0; b < BN / 2; ++b) {
           if ((b & 7) >= C::POLY_PAIRS) continue;
@@ -724,7 +697,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int b = 0; b < BN / 2 && !kSplit; b += EB) {
         if (kPing && kRelease < BN / 2 && b == kRelease) {
           __syncwarp();
-          if (lane == 0) mbar_arrive(bars.tok(t + 1 == NQ ? 0 : t + 1, quarter));
+          if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
         }
         float x[2 * EB];
 #pragma unroll
@@ -755,7 +728,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
       if (kPing && kRelease == BN / 2 && !kSplit) {
         __syncwarp();
-        if (lane == 0) mbar_arrive(bars.tok(t + 1 == NQ ? 0 : t + 1, quarter));
+        if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
       }
       // The previous P V (and the O it accumulates) must be complete before P and O are touched.
       if (!kChunkP && C::P_SEP && gi > 0) {
@@ -784,14 +757,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) r[i] = pk[c * 16 + i];
         tmem_st16(tP + c * 16, r);
-      }
-      if constexpr (BN % 32 == 16) {
-        if (!kChunkP) {
-          uint32_t r[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) r[i] = pk[BN / 2 - 8 + i];
-          tmem_st8(tP + BN / 2 - 8, r);
-        }
       }
       tmem_wait_st();
       tc_fence_before();
@@ -1191,15 +1156,6 @@ sd_status dispatch(const void* q, const void* k, const void* v, void* o, int64_t
       case 64: return launch<Cfg<64, 96, SD_CROSS_NQ, 2, true, false, 0, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
       case 80: return launch<Cfg<80, 96, SD_CROSS_NQ, 2, true, true, 0, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
       default: break;  // dh = 160 already uses 64-key tiles
-    }
-  }
-  // Long query sequences: three query tiles per CTA, whose softmax warps take turns on each SM
-  // sub-partition's special-function unit (narrower key tiles, so that three tiles fit in tensor memory).
-  if (SD_NQ3 && Lq >= 2048) {
-    switch (dh) {
-      case 40: return launch<Cfg<40, 80, 3, 4, true, true, 2, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
-      case 64: return launch<Cfg<64, 64, 3, 4, true, false, 2, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
-      default: break;
     }
   }
   switch (dh) {
