@@ -114,14 +114,6 @@ enum : int { kSplitPublish = 1, kSplitMerge = 2, kSplitAbort = 3 };  // split ha
 #define SD_REGSPLIT 1  // setmaxnreg: 120 registers per helper thread, 192 per softmax thread (two query tiles)
 #endif
 
-#ifndef SD_MMA_BLOCKING
-#define SD_MMA_BLOCKING 0  // MMA issuers in a fixed order behind suspending waits instead of polling
-#endif
-
-#ifndef SD_EXP_SPLIT
-#define SD_EXP_SPLIT 0  // 1: special-function pairs before the token hand-off, polynomial pairs after (slower)
-#endif
-
 #ifndef SD_PINGPONG
 #define SD_PINGPONG 1  // alternate the two query tiles' exp2 phases on each SM sub-partition
 #endif
@@ -434,52 +426,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       bool ok = true;
       long long t_idle = clock64();
       uint32_t spins = 0;
-      // Blocking variant: the fixed order S_0, then S_{g+1} (the softmax releases S_g right after
-      // reading it) before P_g V_g, each behind suspending mbarrier waits instead of polling, so an
-      // idle issuer takes no issue slots from the softmax warps of its sub-partition.
-      constexpr bool kBlocking = SD_MMA_BLOCKING && C::P_SEP;
-      if constexpr (kBlocking) {
-        auto do_qk = [&]() -> bool {
-          const int qb = nseg_q % C::QBUF;
-          if (jq == 0 && !wait_bar(bars.q_full(qb), (nseg_q / C::QBUF) & 1, abort_flag, err)) return false;
-          if (!wait_bar(bars.k_full(gq % STAGES), (gq / STAGES) & 1, abort_flag, err)) return false;
-          if (gq > 0 && !wait_bar(bars.s_free(t), (gq - 1) & 1, abort_flag, err)) return false;
-          tc_fence_after();
-          tq = sbase + C::Q_OFF + (qb * NQ + t) * C::Q_TILE_BYTES;
-          issue_qk(gq % STAGES);
-          mma_commit(bars.s_full(t));
-          ++gq;
-          if (++jq == sq.ke - sq.kb) {
-            mma_commit(bars.q_empty(qb));
-            have_q = next_seg(uq, u1, nkv, sq);
-            jq = 0;
-            ++nseg_q;
-          }
-          return true;
-        };
-        auto do_pv = [&]() -> bool {
-          if (!wait_bar(bars.p_full(t), gp & 1, abort_flag, err)) return false;
-          if (!wait_bar(C::L_IN_V ? bars.v_ready(gp % STAGES) : bars.v_full(gp % STAGES), (gp / STAGES) & 1,
-                        abort_flag, err))
-            return false;
-          tc_fence_after();
-          issue_pv(gp % STAGES, jp == 0);
-          mma_commit(bars.o_done(t));
-          mma_commit(bars.kv_empty(gp % STAGES));
-          ++gp;
-          if (++jp == sp.ke - sp.kb) {
-            have_p = next_seg(up, u1, nkv, sp);
-            jp = 0;
-          }
-          return true;
-        };
-        if (have_q) ok = do_qk();
-        while (ok && have_p) {
-          if (have_q && !do_qk()) break;
-          if (!do_pv()) break;
-        }
-        have_p = false;
-      }
       while (ok && have_p) {
         const bool can_pv = gp < gq && mbar_test_wait(bars.p_full(t), gp & 1) &&
                             mbar_test_wait(C::L_IN_V ? bars.v_ready(gp % STAGES) : bars.v_full(gp % STAGES),
@@ -667,35 +613,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // overlaps the rest of this one (two warps keep the special-function unit busier than one).
       constexpr int kRel = SD_PING_RELEASE >= 0 ? SD_PING_RELEASE : C::PING_RELEASE;
       constexpr int kRelease = kRel > BN / 2 ? BN / 2 : kRel / EB * EB;
-      // Split order: the special-function-unit pairs first, then the token, then the FMA-pipe
-      // polynomial pairs, so that this warp's polynomial work overlaps the partner warp's
-      // special-function phase instead of lengthening the phase that holds the token.
-      constexpr bool kSplit = SD_EXP_SPLIT && kPing && C::POLY_PAIRS > 0 && !kChunkP;
-      if constexpr (kSplit) {
 #pragma unroll
-        for (int b = 0; b < BN / 2; ++b) {
-          if ((b & 7) < C::POLY_PAIRS) continue;
-          float x0, x1;
-          fma2(x0, x1, sv[2 * b], sv[2 * b + 1], scale_log2, scale_log2, neg_m, neg_m);
-          x0 = ex2_approx(x0);
-          x1 = ex2_approx(x1);
-          if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x0, x1);
-          pk[b] = C::F16 ? pack_f16x2(x0, x1) : pack_bf16x2(x0, x1);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
-#pragma unroll
-        for (int b = 0; b < BN / 2; ++b) {
-          if ((b & 7) >= C::POLY_PAIRS) continue;
-          float x0, x1;
-          fma2(x0, x1, sv[2 * b], sv[2 * b + 1], scale_log2, scale_log2, neg_m, neg_m);
-          exp2_poly2(x0, x1, x0, x1);
-          if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x0, x1);
-          pk[b] = C::F16 ? pack_f16x2(x0, x1) : pack_bf16x2(x0, x1);
-        }
-      }
-#pragma unroll
-      for (int b = 0; b < BN / 2 && !kSplit; b += EB) {
+      for (int b = 0; b < BN / 2; b += EB) {
         if (kPing && kRelease < BN / 2 && b == kRelease) {
           __syncwarp();
           if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
@@ -727,7 +646,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
       }
       if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
-      if (kPing && kRelease == BN / 2 && !kSplit) {
+      if (kPing && kRelease == BN / 2) {
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
       }
