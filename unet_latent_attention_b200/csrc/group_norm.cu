@@ -33,6 +33,7 @@ namespace cg = cooperative_groups;
 namespace {
 
 constexpr int kThreads = 256;  // streaming path
+constexpr int kMaxGroupChannels = 128;  // resident path: channels per group staged in shared memory
 constexpr int kMaxWarps = 32;
 constexpr int kMaxCluster = 8;
 constexpr int kMaxItems = 16;  // float4 per thread on the resident path
@@ -58,6 +59,30 @@ __device__ __forceinline__ Stats merge(Stats a, Stats b) {
 __device__ __forceinline__ Stats shfl_down(Stats s, int off) {
   return Stats{__shfl_down_sync(0xffffffffu, s.n, off), __shfl_down_sync(0xffffffffu, s.mean, off),
                __shfl_down_sync(0xffffffffu, s.m2, off)};
+}
+
+// The same merge with the approximate division (2 ulp): on the resident path's critical chain
+// (the statistics are complete only when the last of a cluster's loads lands, and the stores wait
+// for them), so its latency matters more than the last bit of the weight.
+__device__ __forceinline__ Stats merge_fast(Stats a, Stats b) {
+  const float n = a.n + b.n;
+  if (n == 0.f) return a;
+  const float d = b.mean - a.mean;
+  const float fb = __fdividef(b.n, n);
+  return Stats{n, fmaf(d, fb, a.mean), a.m2 + b.m2 + d * d * a.n * fb};
+}
+
+// Merges the triples of lanes [0, n) (n a power of two, at most 32) toward lane 0 in a fixed tree
+// and returns lane 0's result in every lane: every warp that runs it on the same inputs gets the
+// same bits.
+__device__ __forceinline__ Stats warp_tree_merge(Stats st, int n) {
+  const int lane = threadIdx.x & 31;
+  for (int off = n >> 1; off > 0; off >>= 1) {
+    const Stats o = shfl_down(st, off);
+    if (lane + off < n) st = merge_fast(st, o);
+  }
+  return Stats{__shfl_sync(0xffffffffu, st.n, 0), __shfl_sync(0xffffffffu, st.mean, 0),
+               __shfl_sync(0xffffffffu, st.m2, 0)};
 }
 
 // Exact statistics of four values (two sweeps over registers).
@@ -145,6 +170,43 @@ __device__ __forceinline__ void cluster_group_stats(Stats st, float eps, float* 
   __syncthreads();
 }
 
+// Resident path's statistics, then the per-channel affine of the group: the thread's triple is
+// merged over its warp (shuffles), the warps' triples by warp 0 (one shuffle tree), and warp 0's
+// lanes push the CTA's triple into slot `rank` of every peer's shared memory at once; after one
+// cluster barrier warp 0 merges the slots in a fixed tree (so every CTA of the cluster obtains the
+// same bits) and writes a_c = rstd * gamma_c and b_c = beta_c - mean * a_c for the group's cpg
+// channels (gamma and beta already staged in s_a / s_b) into shared memory.
+__device__ __forceinline__ void cluster_group_affine(Stats st, float eps, int cpg, float* s_a, float* s_b,
+                                                     Stats* s_warp, Stats* s_all) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const Stats o = shfl_down(st, off);
+    if (lane + off < 32) st = merge_fast(st, o);
+  }
+  if (lane == 0) s_warp[warp] = st;
+  __syncthreads();
+  const int cs = static_cast<int>(cluster.num_blocks());
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;  // 8, 16 or 32
+    const Stats a = warp_tree_merge(lane < nw ? s_warp[lane] : Stats{0.f, 0.f, 0.f}, nw);
+    if (lane < cs) *cluster.map_shared_rank(&s_all[cluster.block_rank()], lane) = a;
+  }
+  cluster.sync();  // release/acquire: every peer's slot write is visible
+  if (warp == 0) {
+    const Stats a = warp_tree_merge(lane < cs ? s_all[lane] : Stats{0.f, 0.f, 0.f}, cs);
+    const float var = a.n > 0.f ? fmaxf(a.m2 / a.n, 0.f) : 0.f;
+    const float rstd = rsqrtf(var + eps);
+    for (int c = lane; c < cpg; c += 32) {
+      const float ac = rstd * s_a[c];
+      s_b[c] = fmaf(-a.mean, ac, s_b[c]);
+      s_a[c] = ac;
+    }
+  }
+  __syncthreads();
+}
+
 // Resident path: one cluster of `cs` CTAs per (b, g); CTA `rank` owns elements
 // [rank*chunk, (rank+1)*chunk) of the group, chunk a multiple of 4, held in registers.
 // 512-thread CTAs with up to 10 float4 per thread are compiled for 2 resident CTAs per SM (64
@@ -155,14 +217,21 @@ __device__ __forceinline__ void cluster_group_stats(Stats st, float eps, float* 
 #define SD_GN_MINB 1
 #endif
 
+// Resident CTAs per SM the register budget is compiled for: enough CTAs in flight to cover the
+// load latency (256-thread CTAs: 4 with at most 5 float4 per thread, 3 with at most 10).
+constexpr int gn_min_blocks(int items, int threads) {
+  return threads == 512 ? ((SD_GN_MINB && items <= 10) ? 2 : 1)
+                        : threads == 256 ? (items <= 5 ? 4 : items <= 10 ? 3 : 1) : 1;
+}
+
 template <int ITEMS, int THREADS, int EPI>
-__global__ void __launch_bounds__(THREADS, (SD_GN_MINB && THREADS == 512 && ITEMS <= 10) ? 2 : 1) gn_resident(const float* x, const float* __restrict__ gamma,
+__global__ void __launch_bounds__(THREADS, gn_min_blocks(ITEMS, THREADS)) gn_resident(const float* x, const float* __restrict__ gamma,
                                                         const float* __restrict__ beta, void* y,
                                                         int group_elems, int chunk, int hw, int cpg, int groups,
                                                         float eps) {
   __shared__ Stats s_warp[THREADS / 32];
   __shared__ Stats s_all[kMaxCluster];
-  __shared__ float s_mean, s_rstd;
+  __shared__ float s_a[kMaxGroupChannels], s_b[kMaxGroupChannels];
   sd::grid_dep_wait();
   sd::grid_dep_launch();
   cg::cluster_group cluster = cg::this_cluster();
@@ -178,6 +247,11 @@ __global__ void __launch_bounds__(THREADS, (SD_GN_MINB && THREADS == 512 && ITEM
   for (int i = 0; i < ITEMS; ++i) {
     const int idx = threadIdx.x + i * THREADS;
     v[i] = idx < n4 ? ld_stream(xg + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // the group's gamma and beta, staged while the loads above are in flight
+  for (int c = threadIdx.x; c < cpg; c += THREADS) {
+    s_a[c] = __ldg(gamma + g * cpg + c);
+    s_b[c] = __ldg(beta + g * cpg + c);
   }
   // Thread triple: exact mean of its values, then M2 about it.
   float sum = 0.f, cnt = 0.f;
@@ -196,20 +270,28 @@ __global__ void __launch_bounds__(THREADS, (SD_GN_MINB && THREADS == 512 && ITEM
       st.m2 += a * a + b * b + c * c + d * d;
     }
   }
-  cluster_group_stats(st, eps, &s_mean, &s_rstd, s_warp, s_all);
-  const float mean = s_mean, rstd = s_rstd;
+  cluster_group_affine(st, eps, cpg, s_a, s_b, s_warp, s_all);
 
   const int64_t base4 = base >> 2;  // base is a multiple of 4 (chunk and group_elems are)
-  const int e0 = rank * chunk;
+  // Channel (within the group) of this thread's item i, element rank * chunk + 4 (tid + i THREADS):
+  // one division here, then a step of 4 THREADS elements per item (hw % 4 == 0: a float4 never
+  // straddles channels).
+  const int e_first = rank * chunk + 4 * static_cast<int>(threadIdx.x);
+  int ch = e_first / hw, rem = e_first - ch * hw;
+  const int step_c = 4 * THREADS / hw, step_r = 4 * THREADS - step_c * hw;
 #pragma unroll
   for (int i = 0; i < ITEMS; ++i) {
     const int idx = threadIdx.x + i * THREADS;
     if (idx < n4) {
-      const int c = g * cpg + (e0 + idx * 4) / hw;  // hw % 4 == 0: a float4 never straddles channels
-      const float a = rstd * __ldg(gamma + c);
-      const float b = fmaf(-mean, a, __ldg(beta + c));
+      const float a = s_a[ch], b = s_b[ch];
       store4<EPI>(y, base4 + idx, make_float4(fmaf(v[i].x, a, b), fmaf(v[i].y, a, b), fmaf(v[i].z, a, b),
                                               fmaf(v[i].w, a, b)));
+    }
+    ch += step_c;
+    rem += step_r;
+    if (rem >= hw) {
+      rem -= hw;
+      ++ch;
     }
   }
 }
@@ -316,7 +398,7 @@ sd_status group_norm_impl(const char* name, const float* x, const float* gamma, 
   // Policy (measured on the SD shapes): the smallest cluster and CTA size that still put about
   // one CTA on every SM.
   const bool y_vec = EPI == kSiluBf16 ? (reinterpret_cast<uintptr_t>(y) & 7u) == 0 : sd::aligned16(y);
-  const bool vec_ok = hw % 4 == 0 && sd::aligned16(x) && y_vec;
+  const bool vec_ok = hw % 4 == 0 && cpg <= kMaxGroupChannels && sd::aligned16(x) && y_vec;
   int cs = 0, threads = 0;
   if (vec_ok && SD_GN_POLICY == 0) {
     // First choice (measured on the inner UNet levels): 256-thread CTAs in the smallest cluster that
