@@ -575,18 +575,38 @@ def bench_extra(sdk, dev, hbm):
     return out
 
 
+def _packed(like: dict, keys, **alloc):
+    """One contiguous byte buffer holding a tensor per key (each at a 256-byte aligned offset) and the
+    views into it: a step's inputs (or outputs) then cross the host link as one copy."""
+    import torch
+    offs, n = {}, 0
+    for k in keys:
+        offs[k] = n
+        n += (like[k].numel() * like[k].element_size() + 255) // 256 * 256
+    blob = torch.empty(n, dtype=torch.uint8, **alloc)
+    views = {k: blob[offs[k]:offs[k] + like[k].numel() * like[k].element_size()].view(like[k].dtype).view(like[k].shape)
+             for k in keys}
+    return blob, views
+
+
 def bench_e2e(args, sdk, S, g, a_t, a_p, w, flops_step, world, dev):
     """Same step through the public API with host buffers: every step copies all of its inputs from
     pinned host memory to the device, runs the four launches and copies every output back, all inside
-    the timed region. Two device buffer sets and three streams let step i's inputs travel while step
-    i-1 computes and step i-2's outputs travel back (the host link carries both directions at once);
-    the serial form (one stream) is reported beside it."""
+    the timed region. The inputs sit in one pinned buffer and the outputs in another, so each
+    direction is one copy per step. Two device buffer sets and three streams let step i's inputs
+    travel while step i-1 computes and step i-2's outputs travel back (the host link carries both
+    directions at once); the serial form (one stream) is reported beside it."""
     import torch
-    host_in = {k: S[k].cpu().pin_memory() for k in INPUT_KEYS}
-    host_out = {k: torch.empty(S[k].shape, dtype=S[k].dtype, pin_memory=True) for k in OUTPUT_KEYS}
-    bufs = [{k: torch.empty_like(S[k]) for k in INPUT_KEYS + OUTPUT_KEYS} for _ in range(2)]
-    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    h_in, host_in = _packed(S, INPUT_KEYS, pin_memory=True)
+    for k in INPUT_KEYS:
+        host_in[k].copy_(S[k].cpu())
+    h_out, host_out = _packed(S, OUTPUT_KEYS, pin_memory=True)
+    bufs = []
+    for _ in range(2):
+        d_in, vin = _packed(S, INPUT_KEYS, device=dev)
+        d_out, vout = _packed(S, OUTPUT_KEYS, device=dev)
+        bufs.append((d_in, d_out, {**vin, **vout}))
+    h2d, d2h = h_in.numel(), h_out.numel()  # bytes copied per step (tensors plus alignment padding)
     n = max(3, min(args.steps, 50))
     s_in, s_c, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
 
@@ -597,12 +617,11 @@ def bench_e2e(args, sdk, S, g, a_t, a_p, w, flops_step, world, dev):
         if e0 is not None:
             e0.record(s_in)
         for i in range(steps):
-            b = bufs[i % 2]
+            d_in, d_out, b = bufs[i % 2]
             with torch.cuda.stream(s_in):
                 if i >= 2:
                     s_in.wait_event(ev_c[i - 2])  # step i-2 has finished reading this set's inputs
-                for k in INPUT_KEYS:
-                    b[k].copy_(host_in[k], non_blocking=True)
+                d_in.copy_(h_in, non_blocking=True)
                 ev_in[i].record(s_in)
             with torch.cuda.stream(s_c):
                 s_c.wait_event(ev_in[i])
@@ -612,21 +631,18 @@ def bench_e2e(args, sdk, S, g, a_t, a_p, w, flops_step, world, dev):
                 ev_c[i].record(s_c)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_c[i])
-                for k in OUTPUT_KEYS:
-                    host_out[k].copy_(b[k], non_blocking=True)
+                h_out.copy_(d_out, non_blocking=True)
                 ev_out[i].record(s_out)
         if e1 is not None:
             s_out.wait_event(ev_out[-1])
             e1.record(s_out)
 
     def serial(steps):
-        b = bufs[0]
+        d_in, d_out, b = bufs[0]
         for _ in range(steps):
-            for k in INPUT_KEYS:
-                b[k].copy_(host_in[k], non_blocking=True)
+            d_in.copy_(h_in, non_blocking=True)
             run_step(sdk, b, g, a_t, a_p, w)
-            for k in OUTPUT_KEYS:
-                host_out[k].copy_(b[k], non_blocking=True)
+            h_out.copy_(d_out, non_blocking=True)
 
     pipelined(3)
     serial(3)
@@ -649,7 +665,8 @@ def bench_e2e(args, sdk, S, g, a_t, a_p, w, flops_step, world, dev):
     sdk.sd_device_status()
     return {"value": whole_job_tflops(flops_step, n, world, ms), "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms / n, "steps": n,
-            "form": "two buffer sets, copy-in / compute / copy-out streams",
+            "form": "inputs and outputs each one pinned buffer; two device buffer sets, copy-in / compute / "
+                    "copy-out streams",
             "serial": {"value": whole_job_tflops(flops_step, n, world, ms_serial), "ms_per_step": ms_serial / n}}
 
 

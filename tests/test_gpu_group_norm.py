@@ -33,7 +33,11 @@ def test_workload_shapes(cuda, wid, label, shape):
 
 @pytest.mark.parametrize("shape,groups", [((1, 32, 7, 9), 32), ((2, 64, 3, 3), 32), ((3, 8, 5, 4), 1),
                                           ((2, 12, 4, 4), 12), ((1, 64, 128, 128), 2), ((2, 320, 1, 1), 32),
-                                          ((1, 4, 257, 3), 2)])
+                                          ((1, 4, 257, 3), 2),
+                                          # channels per group staged in shared memory: 48, 96 and the
+                                          # limit 128 (resident path); 160 and 256 take the streaming path
+                                          ((1, 48, 32, 32), 1), ((2, 96, 16, 16), 1), ((1, 128, 8, 8), 1),
+                                          ((2, 640, 4, 4), 4), ((1, 256, 8, 8), 1)])
 def test_odd_shapes(cuda, shape, groups):
     x = si.normal(shape, 500 + sum(shape))
     C = shape[1]
