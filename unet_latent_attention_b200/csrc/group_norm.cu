@@ -10,15 +10,15 @@
 //  * Statistics stay in fp32 but are merged as (count, mean, M2) triples with the pairwise update
 //    of Chan, Golub and LeVeque (1979) -- warp shuffles, then shared memory across warps, then
 //    distributed shared memory across the cluster -- instead of sum / sum-of-squares, which
-//    cancels when |mean| >> std. Every CTA of a cluster merges the per-CTA triples in rank order,
-//    so all of them obtain bit-identical statistics.
+//    cancels when |mean| >> std. Every CTA of a cluster merges the per-CTA triples in one fixed
+//    tree, so all of them obtain bit-identical statistics.
 //  * The tail is fused: y = x * a_c + b_c with a_c = rstd * gamma[c], b_c = beta[c] - mean * a_c.
 //    sd_group_norm_silu adds the SiLU activation, v * sigmoid(v), that follows GroupNorm in the
 //    UNet's residual blocks (the page's GroupNorm + SiLU single-kernel fusion, §9), with an fp32 or
 //    bf16 output.
 //
-// Shapes the resident path cannot hold (groups above 8 x 16384 elements, H*W not a multiple of 4,
-// pointers not 16-byte aligned) take the streaming path: the same cluster merge, but each CTA
+// Shapes the resident path cannot hold (groups above 8 x 16384 elements, more than 128 channels per
+// group, H*W not a multiple of 4, pointers not 16-byte aligned) take the streaming path: the same cluster merge, but each CTA
 // sweeps its part twice (statistics, then normalise), so x is read twice (the second time mostly
 // from L2). Neither path uses global scratch memory.
 #include <cooperative_groups.h>
