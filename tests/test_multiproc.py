@@ -54,3 +54,25 @@ def test_single_process_reduce_is_identity():
     import torch
     import bench
     assert bench.reduce_max([1.5, 2.5], torch.device("cpu")) == [1.5, 2.5]
+
+
+def test_packed_step_buffers_hold_every_tensor_aligned_and_apart():
+    # the end-to-end step moves a step's inputs (outputs) as one buffer: every tensor must be a
+    # view at a 256-byte aligned offset, of its own shape and type, and no two views may overlap
+    import torch
+    import bench
+    like = {"q": torch.zeros(2, 8, 33, 40, dtype=torch.bfloat16), "x": torch.zeros(2, 5, 3, 3),
+            "g": torch.zeros(7), "lat": torch.zeros(1, 4, 8, 8)}
+    blob, views = bench._packed(like, list(like))
+    spans = []
+    for k, t in like.items():
+        v = views[k]
+        assert v.shape == t.shape and v.dtype == t.dtype and v.is_contiguous()
+        off = v.data_ptr() - blob.data_ptr()
+        assert off % 256 == 0
+        spans.append((off, off + v.numel() * v.element_size()))
+        v.fill_(1)
+    spans.sort()
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+    assert spans[-1][1] <= blob.numel()
+    assert float(views["q"].float().sum()) == like["q"].numel()
