@@ -400,7 +400,18 @@ sd_status group_norm_impl(const char* name, const float* x, const float* gamma, 
   const bool y_vec = EPI == kSiluBf16 ? (reinterpret_cast<uintptr_t>(y) & 7u) == 0 : sd::aligned16(y);
   const bool vec_ok = hw % 4 == 0 && cpg <= kMaxGroupChannels && sd::aligned16(x) && y_vec;
   int cs = 0, threads = 0;
-  if (vec_ok && SD_GN_POLICY == 0) {
+  if (vec_ok && SD_GN_POLICY == 0 && group_elems % 16 == 0) {
+    // Groups of 40960-81920 elements (the SD/SDXL top levels, 10 or 20 channels of 64 x 64): clusters
+    // of 4 CTAs x 512 threads with 5-10 float4 per thread, two CTAs per SM -- measured faster than
+    // 8 x 256 ([2,320,64,64] 7.7 -> 7.5 us, [2,640,64,64] 13.7 -> 11.7, [16,640,64,64] 66.8 -> 61.0).
+    const int64_t sms = sd::sm_count();
+    const int64_t need = (group_elems / 4 / 4 + 511) / 512;
+    if (need >= 5 && need <= 10 && n_groups * 4 >= sms) {
+      cs = 4;
+      threads = 512;
+    }
+  }
+  if (vec_ok && SD_GN_POLICY == 0 && !cs) {
     // First choice (measured on the inner UNet levels): 256-thread CTAs in the smallest cluster that
     // still gives one CTA per SM, if that holds at most 6 float4 per thread -- half as many CTAs and
     // cheaper cluster barriers ([2,640,32,32] 5.9 -> 5.1 us, [2,1280,16,16] 5.7 -> 4.0 us). With
