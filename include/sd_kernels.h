@@ -59,7 +59,7 @@ typedef enum sd_status {
  *  groups : must divide C (SD_ERR_INVALID_ARG otherwise); 32 in Stable Diffusion.
  *  eps    : > 0 and finite (1e-5 in Stable Diffusion).
  * Statistics are accumulated in fp32 with a pairwise (Chan et al.) merge. Groups of up to
- * 131072 elements and at most 128 channels, with H*W % 4 == 0 and 16-byte aligned x and y, are
+ * 262144 elements and at most 128 channels, with H*W % 4 == 0 and 16-byte aligned x and y, are
  * read from HBM once (a thread-block cluster of up to 8 CTAs holds the group in registers); other
  * shapes take a streaming path of the same single launch that reads x twice. No global scratch
  * is used.

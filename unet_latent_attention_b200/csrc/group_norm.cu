@@ -17,7 +17,7 @@
 //    UNet's residual blocks (the page's GroupNorm + SiLU single-kernel fusion, §9), with an fp32 or
 //    bf16 output.
 //
-// Shapes the resident path cannot hold (groups above 8 x 16384 elements, more than 128 channels per
+// Shapes the resident path cannot hold (groups above 8 x 32768 elements, more than 128 channels per
 // group, H*W not a multiple of 4, pointers not 16-byte aligned) take the streaming path: the same cluster merge, but each CTA
 // sweeps its part twice (statistics, then normalise), so x is read twice (the second time mostly
 // from L2). Neither path uses global scratch memory.
