@@ -489,7 +489,7 @@ def bench_extra(sdk, dev, hbm):
     workload (DDIM, DPM-Solver++(2M), third order) as CUDA graphs over independent loop sets whose
     latents and noise predictions exceed 2.5x L2 in total; a size sweep of GroupNorm (+SiLU),
     CFG+DDIM and CFG+DPM-Solver++ up to buffers far larger than L2 with rotating inputs; and
-    cross-attention with longer text contexts and fp16 attention."""
+    cross-attention with longer text contexts, fp16 attention and the [B, L, heads, dh] layout."""
     import torch
     out = {}
     lat = si.WORKLOADS[5].latent
@@ -561,16 +561,28 @@ def bench_extra(sdk, dev, hbm):
         for k in ("frac_tensor", "peak_tensor"):
             long[-1].pop(k)
     out["cross_attention_text_length"] = long
-    f16 = []
-    for Lk in (4096, 77):  # fp16 tensors on the SD1.5 512x512 self- and cross-attention shapes
-        nsets = 12
+    f16, blhd = [], []
+    for Lk in (4096, 77):  # the SD1.5 512x512 self- and cross-attention shapes
+        flops = 4 * 2 * 8 * 4096 * Lk * 40
+        nsets = _n_rotating(2 * (2 * 2 * 8 * 4096 * 40 + 2 * 2 * 8 * Lk * 40), cap=64)
+        # fp16 tensors, [B, heads, L, dh]
         sets = [tuple(torch.randn(2, 8, L, 40, device=dev, dtype=torch.float16) for L in (4096, Lk, Lk))
                 for _ in range(nsets)]
         outs = [torch.empty_like(s[0]) for s in sets]
         us, _ = _graph_time_us(lambda i: sdk.sd_attention(*sets[i % nsets], out=outs[i % nsets]), nsets, dev)
-        f16.append({"shape": [2, 8, 4096, Lk, 40], "us": us, "TFLOP/s": 4 * 2 * 8 * 4096 * Lk * 40 / (us * 1e-6) / 1e12})
+        f16.append({"shape": [2, 8, 4096, Lk, 40], "us": us, "TFLOP/s": flops / (us * 1e-6) / 1e12, "rotating_sets": nsets})
+        del sets, outs
+        # bf16 tensors in the [B, L, heads, dh] layout a fused QKV projection writes
+        sets = [tuple(torch.randn(2, L, 8, 40, device=dev, dtype=torch.bfloat16) for L in (4096, Lk, Lk))
+                for _ in range(nsets)]
+        outs = [torch.empty_like(s[0]) for s in sets]
+        us, _ = _graph_time_us(lambda i: sdk.sd_attention(*sets[i % nsets], out=outs[i % nsets], layout="blhd"),
+                               nsets, dev)
+        blhd.append({"shape": [2, 4096, 8, 40], "Lk": Lk, "us": us, "TFLOP/s": flops / (us * 1e-6) / 1e12,
+                     "rotating_sets": nsets})
         del sets, outs
     out["attention_fp16"] = f16
+    out["attention_blhd"] = blhd
     torch.cuda.empty_cache()
     return out
 
