@@ -151,6 +151,15 @@ def test_split_items_after_other_head_dims(cuda):
         _check(o, oracle.attention(q, k, v))
 
 
+@pytest.mark.parametrize("dh,B,heads,Lq,Lk", [(40, 1, 1, 2048, 4096), (64, 1, 2, 700, 3000), (80, 1, 1, 256, 2000)])
+def test_fewer_items_than_sms(cuda, dh, B, heads, Lq, Lk):
+    # a few long items: the grid shrinks to one CTA per item (no split), each streaming many K/V
+    # tiles with a ragged last one
+    q, k, v = _qkv(B, heads, Lq, Lk, dh, 9500 + dh + Lq + Lk)
+    o = _run(q, k, v, cuda)
+    _check(o, oracle.attention(q, k, v))
+
+
 def test_repeated_launches_reuse_the_hand_off_flags(cuda):
     # the split hand-off flags must return to zero after every launch (graph replays rely on it)
     q, k, v = _qkv(2, 80, 256, 640, 40, 9100)
