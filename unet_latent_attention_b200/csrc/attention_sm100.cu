@@ -130,6 +130,10 @@ enum : int { kSplitPublish = 1, kSplitMerge = 2, kSplitAbort = 3 };  // split ha
 #define SD_PING_SHORT 1  // ping-pong also for the single 96-key tile of short key sequences
 #endif
 
+#ifndef SD_SMALL_NQ1
+#define SD_SMALL_NQ1 1  // one query tile per CTA while there are at most this many query tiles per SM
+#endif
+
 #ifndef SD_STAGES_SMALL
 #define SD_STAGES_SMALL 4  // K/V ring depth for head dims <= 64 (one 16 KB K and V tile per stage)
 #endif
@@ -1076,6 +1080,16 @@ sd_status dispatch(const void* q, const void* k, const void* v, void* o, int64_t
       case 64: return launch<Cfg<64, 96, SD_CROSS_NQ, 2, true, false, 0, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
       case 80: return launch<Cfg<80, 96, SD_CROSS_NQ, 2, true, true, 0, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
       default: break;  // dh = 160 already uses 64-key tiles
+    }
+  }
+  // Few query tiles (every tile can have an SM of its own): one query tile per CTA, so that twice as
+  // many SMs share the work.
+  if (SD_SMALL_NQ1 && BH * ((Lq + BM - 1) / BM) <= SD_SMALL_NQ1 * sd::sm_count()) {
+    switch (dh) {
+      case 40: return launch<Cfg<40, 128, 1, 4, true, true, 2, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+      case 64: return launch<Cfg<64, 128, 1, 4, true, false, 2, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+      case 80: return launch<Cfg<80, 128, 1, 2, false, true, 0, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+      default: break;
     }
   }
   switch (dh) {
