@@ -1083,12 +1083,14 @@ sd_status dispatch(const void* q, const void* k, const void* v, void* o, int64_t
     }
   }
   // Few query tiles (every tile can have an SM of its own): one query tile per CTA, so that twice as
-  // many SMs share the work.
+  // many SMs share the work. With one tile the dh 80 tile's S, P and O fit 512 tensor-memory columns
+  // side by side, so the next S no longer waits for P V (measured 20.7 -> 16.8 us at [2,8,1024,1024,80]
+  // with 2 of 8 exp2 pairs on the FMA pipe).
   if (SD_SMALL_NQ1 && BH * ((Lq + BM - 1) / BM) <= SD_SMALL_NQ1 * sd::sm_count()) {
     switch (dh) {
       case 40: return launch<Cfg<40, 128, 1, 4, true, true, 2, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
       case 64: return launch<Cfg<64, 128, 1, 4, true, false, 2, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
-      case 80: return launch<Cfg<80, 128, 1, 2, false, true, 0, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
+      case 80: return launch<Cfg<80, 128, 1, 2, true, true, 2, F16, BLHD>>(q, k, v, o, BH, Lq, Lk, dh, scale, s, fixed, lay_heads);
       default: break;
     }
   }
