@@ -386,6 +386,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             wait_bar(bars.v_full(s), (issued[s] - 1) & 1, abort_flag, err, false);
         }
     }
+    __syncwarp();  // lanes 1-31 wait for lane 0 here: the warp meets the CTA barrier below as a whole
   } else if (warp == 1 || (NQ == 2 && warp == 2)) {
     // ------------------------------------------------------------------ MMA issuer of one tile
     // One issuing warp per query tile: a tcgen05.mma occupies its issuing thread for tens to
@@ -749,11 +750,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         ok = false;
         break;
       }
+      // Slot layout: for each warp of 32 rows, float4 i of all 32 rows is one contiguous 512-byte
+      // run (coalesced writes and reads: a row-major slot made every access of a warp touch 32
+      // lines), then (m, l) of every row.
       if (*dec == kSplitPublish) {
-        float4* dst = reinterpret_cast<float4*>(slot + static_cast<size_t>(slot_row) * C::NPV);
+        float4* dst = reinterpret_cast<float4*>(slot) + (slot_row >> 5) * (C::NPV / 4) * 32 + lane;
 #pragma unroll
         for (int i = 0; i < C::NPV / 4; ++i)
-          dst[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
+          dst[i * 32] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
         reinterpret_cast<float2*>(slot + NQ * BM * C::NPV)[slot_row] = make_float2(m_run, lsum);
         // Every softmax thread arrives (release, CTA scope); the leader waits for all of them, then
         // makes the slot visible device-wide with one fence and marks it complete.
@@ -775,7 +779,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (leader_warp && lane == 0) atomicExch(cnt, 0u);  // both pieces are done with the counter
       // Merge in one fixed order, O = O_head * 2^(m_head - m) + O_tail * 2^(m_tail - m), so the result
       // is the same bit for bit whichever piece merges. The slot is read through L2 only.
-      const float4* src = reinterpret_cast<const float4*>(slot + static_cast<size_t>(slot_row) * C::NPV);
+      const float4* src = reinterpret_cast<const float4*>(slot) + (slot_row >> 5) * (C::NPV / 4) * 32 + lane;
       const float2 ml = __ldcg(reinterpret_cast<const float2*>(slot + NQ * BM * C::NPV) + slot_row);
       const float m_head = kind ? m_run : ml.x, m_tail = kind ? ml.x : m_run;
       const float m_all = fmaxf(m_head, m_tail);
@@ -785,7 +789,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       };
 #pragma unroll
       for (int i = 0; i < C::NPV / 4; ++i) {
-        const float4 o4 = __ldcg(src + i);
+        const float4 o4 = __ldcg(src + i * 32);
         ov[4 * i] = comb(ov[4 * i], o4.x);
         ov[4 * i + 1] = comb(ov[4 * i + 1], o4.y);
         ov[4 * i + 2] = comb(ov[4 * i + 2], o4.z);
