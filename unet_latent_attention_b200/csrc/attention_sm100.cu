@@ -430,6 +430,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       int nseg_q = 0, jq = 0, jp = 0, gq = 0, gp = 0;
       bool ok = true;
       long long t_idle = clock64();
+      // The last tile's issuer also decides the split hand-off (below): it claims a split piece's
+      // slot when it issues the piece's last S, so the atomic's round trip overlaps that tile's
+      // softmax, and publishes the decision to the softmax warps when it issues the last P V.
+      const bool decider = t == NQ - 1;
+      unsigned int claim_head = 0u, claim_tail = 0u;
       uint32_t spins = 0;
       while (ok && have_p) {
         const bool can_pv = gp < gq && mbar_test_wait(bars.p_full(t), gp & 1) &&
@@ -442,6 +447,29 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           mma_commit(bars.kv_empty(gp % STAGES));
           ++gp;
           if (++jp == sp.ke - sp.kb) {
+            if (decider && (sp.kb > 0 || sp.ke < nkv)) {
+              const int kind = sp.ke < nkv ? 1 : 0;  // 1: head piece, 0: tail piece
+              const unsigned int old = kind ? claim_head : claim_tail;
+              int d = old == 0u ? kSplitPublish : kSplitMerge;
+              if (old == 1u) {  // the other piece claimed the slot: wait until it has been completed
+                volatile unsigned int* f = flags + (kind ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) - 1);
+                const long long w0 = clock64();
+                for (uint32_t it = 0; *f != 2u; ++it) {
+                  __nanosleep(32);
+                  if ((it & 63u) == 63u && (*abort_flag || clock64() - w0 > kWaitLimitCycles)) {
+                    if (!*abort_flag) {
+                      *abort_flag = 1;
+                      atomicOr(err, sd::kDevErrTimeout);
+                    }
+                    d = kSplitAbort;
+                    break;
+                  }
+                }
+              }
+              if (d == kSplitMerge) __threadfence();
+              reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 8)[kind] = d;
+              mbar_arrive(bars.split_dec(kind));
+            }
             have_p = next_seg(up, u1, nkv, sp);
             jp = 0;
           }
@@ -459,6 +487,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           mma_commit(bars.s_full(t));
           ++gq;
           if (++jq == sq.ke - sq.kb) {
+            if (decider && (sq.kb > 0 || sq.ke < nkv)) {  // claim: counter 0 -> 1 makes this piece the publisher
+              if ((debug_flags & 2) && sq.ke == nkv) {  // test hook: hold tail pieces back ~50 us (head finishes first)
+                const long long h0 = clock64();
+                while (clock64() - h0 < 100000) __nanosleep(500);
+              }
+              const unsigned int old =
+                  atomicCAS(flags + (sq.ke < nkv ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) - 1), 0u, 1u);
+              if (sq.ke < nkv) claim_head = old;
+              else claim_tail = old;
+            }
             mma_commit(bars.q_empty(qb));  // this tile is done reading the segment's Q
             have_q = next_seg(uq, u1, nkv, sq);
             jq = 0;
@@ -707,44 +745,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (sg.kb > 0 || sg.ke < nkv) {
       // Split item: a head piece (keys [0, k), at the end of CTA c's range) and a tail piece (keys
       // [k, nkv), at the start of CTA c+1's range) share one slot and one counter of boundary c.
-      // Whichever piece finishes first claims the slot (counter 0 -> 1), writes its raw O, m and
-      // l there and marks it complete (-> 2); the other piece merges the two and stores O, then
+      // The piece whose last S = Q K^T is issued first claims the slot (counter 0 -> 1, by the
+      // last tile's MMA issuer, which publishes the decision here), writes its raw O, m and l
+      // there and marks it complete (-> 2); the other piece merges the two and stores O, then
       // resets the counter for the next launch. No CTA ever waits for another CTA to start: the
-      // only cross-CTA wait is the second finisher's wait for a claimed slot to be completed, by a
-      // CTA that is already running and whose write depends on nothing else.
+      // only cross-CTA wait is the other piece's issuer waiting for a claimed slot to be
+      // completed, by a CTA that is already running and whose write depends on nothing else.
       const int kind = sg.ke < nkv ? 1 : 0;  // 1: head piece, 0: tail piece
       const int bnd = kind ? static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x) - 1;
       float* slot = ws + static_cast<size_t>(bnd) * C::SLOT_FLOATS;
       unsigned int* cnt = flags + bnd;
       volatile int* dec = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 8) + kind;
-      const bool leader_warp = warp == C::SOFT_WARP0 + 4 * NQ - 1;  // usually the last to get here
-      if (leader_warp && lane == 0) {
-        if ((debug_flags & 2) && kind == 0) {  // test hook: hold tail pieces back ~50 us (head finishes first)
-          const long long t0 = clock64();
-          while (clock64() - t0 < 100000) __nanosleep(500);
-        }
-        int d = kSplitMerge;
-        if (atomicCAS(cnt, 0u, 1u) == 0u) {
-          d = kSplitPublish;
-        } else {  // the other piece claimed the slot: wait until it has been completed
-          volatile unsigned int* f = cnt;
-          const long long w0 = clock64();
-          for (uint32_t it = 0; *f != 2u; ++it) {
-            __nanosleep(32);
-            if ((it & 63u) == 63u && (*abort_flag || clock64() - w0 > kWaitLimitCycles)) {
-              if (!*abort_flag) {
-                *abort_flag = 1;
-                atomicOr(err, sd::kDevErrTimeout);
-              }
-              d = kSplitAbort;
-              break;
-            }
-          }
-          __threadfence();
-        }
-        *dec = d;
-        mbar_arrive(bars.split_dec(kind));
-      }
+      const bool leader_warp = warp == C::SOFT_WARP0 + 4 * NQ - 1;  // completes a publication
       __syncwarp();
       if (!__all_sync(0xffffffffu, wait_bar(bars.split_dec(kind), 0, abort_flag, err)) || *dec == kSplitAbort) {
         ok = false;
