@@ -8,10 +8,12 @@
 //    cluster of up to 8 CTAs. Each thread loads its part of the group into registers with 16-byte
 //    streaming loads, so HBM is read exactly once (the resident path).
 //  * Statistics stay in fp32 but are merged as (count, mean, M2) triples with the pairwise update
-//    of Chan, Golub and LeVeque (1979) -- warp shuffles, then shared memory across warps, then
-//    distributed shared memory across the cluster -- instead of sum / sum-of-squares, which
-//    cancels when |mean| >> std. Every CTA of a cluster merges the per-CTA triples in one fixed
-//    tree, so all of them obtain bit-identical statistics.
+//    of Chan, Golub and LeVeque (1979) instead of sum / sum-of-squares, which cancels when
+//    |mean| >> std. Resident path: warp shuffles, then every warp sends its triple into every
+//    cluster peer's shared memory with st.async, counted on the peer's mbarrier (no cluster-wide
+//    barrier on the critical path); streaming path: shared memory across warps, then distributed
+//    shared memory across the cluster behind one cluster barrier. Every CTA of a cluster merges
+//    the triples in one fixed order, so all of them obtain bit-identical statistics.
 //  * The tail is fused: y = x * a_c + b_c with a_c = rstd * gamma[c], b_c = beta[c] - mean * a_c.
 //    sd_group_norm_silu adds the SiLU activation, v * sigmoid(v), that follows GroupNorm in the
 //    UNet's residual blocks (the page's GroupNorm + SiLU single-kernel fusion, §9), with an fp32 or
@@ -34,13 +36,57 @@ namespace {
 
 constexpr int kThreads = 256;  // streaming path
 constexpr int kMaxGroupChannels = 128;  // resident path: channels per group staged in shared memory
-constexpr int kMaxWarps = 32;
 constexpr int kMaxCluster = 8;
 constexpr int kMaxItems = 16;  // float4 per thread on the resident path
 
 #ifndef SD_GN_POLICY
 #define SD_GN_POLICY 0
 #endif
+
+// ---------------------------------------------------------------- cluster exchange primitives
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+// The same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t peer_addr(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+// 16-byte store into a peer's shared memory that counts its bytes on the peer's mbarrier.
+__device__ __forceinline__ void st_async_peer(uint32_t dst, float4 v, uint32_t peer_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+               :: "r"(dst), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(peer_bar) : "memory");
+}
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void bar_init_expect(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(bar) : "memory");
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
+               :: "r"(bar), "r"(bytes) : "memory");
+}
+// Waits (acquire, cluster scope) for phase 0 of `bar`; gives up after about a second and reports a
+// timeout in the status word instead of hanging.
+__device__ __forceinline__ void bar_wait_cluster(uint32_t bar, unsigned int* err) {
+  const long long t0 = clock64();
+  for (uint32_t it = 0;; ++it) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(bar) : "memory");
+    if (ok) return;
+    if ((it & 63u) == 63u && clock64() - t0 > 2000000000LL) {
+      atomicOr(err, sd::kDevErrTimeout);
+      return;
+    }
+  }
+}
 
 
 struct Stats {
@@ -170,32 +216,32 @@ __device__ __forceinline__ void cluster_group_stats(Stats st, float eps, float* 
   __syncthreads();
 }
 
-// Resident path's statistics, then the per-channel affine of the group: the thread's triple is
-// merged over its warp (shuffles), the warps' triples by warp 0 (one shuffle tree), and warp 0's
-// lanes push the CTA's triple into slot `rank` of every peer's shared memory at once; after one
-// cluster barrier warp 0 merges the slots in a fixed tree (so every CTA of the cluster obtains the
-// same bits) and writes a_c = rstd * gamma_c and b_c = beta_c - mean * a_c for the group's cpg
-// channels (gamma and beta already staged in s_a / s_b) into shared memory.
-__device__ __forceinline__ void cluster_group_affine(Stats st, float eps, int cpg, float* s_a, float* s_b,
-                                                     Stats* s_warp, Stats* s_all) {
+// Resident path's statistics without a cluster barrier: each warp merges its threads' triples
+// (shuffles) and sends the warp's triple, by st.async, into slot (rank, warp) of every peer's
+// shared memory, where the bytes complete the peer's mbarrier (armed for cs x nw slots before the
+// cluster's arrive at kernel start). Warp 0 waits for its own barrier, merges the cs x nw slots in
+// one fixed order (every CTA obtains the same bits) and writes a_c = rstd * gamma_c and
+// b_c = beta_c - mean * a_c for the group's cpg channels. A CTA receives no slot after its wait,
+// so CTAs may exit without a second cluster-wide sync.
+template <int NW>
+__device__ __forceinline__ void cluster_group_affine_async(Stats st, float eps, int cpg, float* s_a, float* s_b,
+                                                           float4* s_part, uint32_t bar, unsigned int* err) {
   cg::cluster_group cluster = cg::this_cluster();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    const Stats o = shfl_down(st, off);
-    if (lane + off < 32) st = merge_fast(st, o);
-  }
-  if (lane == 0) s_warp[warp] = st;
-  __syncthreads();
-  const int cs = static_cast<int>(cluster.num_blocks());
+  const int cs = static_cast<int>(cluster.num_blocks()), rank = static_cast<int>(cluster.block_rank());
+  const Stats w = warp_tree_merge(st, 32);
+  cluster_wait_acquire();  // every peer's barrier is armed
+  if (lane < cs)
+    st_async_peer(peer_addr(smem_addr(&s_part[rank * NW + warp]), lane), make_float4(w.n, w.mean, w.m2, 0.f),
+                  peer_addr(bar, lane));
   if (warp == 0) {
-    const int nw = blockDim.x >> 5;  // 8, 16 or 32
-    const Stats a = warp_tree_merge(lane < nw ? s_warp[lane] : Stats{0.f, 0.f, 0.f}, nw);
-    if (lane < cs) *cluster.map_shared_rank(&s_all[cluster.block_rank()], lane) = a;
-  }
-  cluster.sync();  // release/acquire: every peer's slot write is visible
-  if (warp == 0) {
-    const Stats a = warp_tree_merge(lane < cs ? s_all[lane] : Stats{0.f, 0.f, 0.f}, cs);
+    bar_wait_cluster(bar, err);
+    Stats a{0.f, 0.f, 0.f};
+    for (int k = lane; k < cs * NW; k += 32) {
+      const float4 p = s_part[k];
+      a = merge_fast(a, Stats{p.x, p.y, p.z});
+    }
+    a = warp_tree_merge(a, 32);
     const float var = a.n > 0.f ? fmaxf(a.m2 / a.n, 0.f) : 0.f;
     const float rstd = rsqrtf(var + eps);
     for (int c = lane; c < cpg; c += 32) {
@@ -228,13 +274,18 @@ template <int ITEMS, int THREADS, int EPI>
 __global__ void __launch_bounds__(THREADS, gn_min_blocks(ITEMS, THREADS)) gn_resident(const float* x, const float* __restrict__ gamma,
                                                         const float* __restrict__ beta, void* y,
                                                         int group_elems, int chunk, int hw, int cpg, int groups,
-                                                        float eps) {
-  __shared__ Stats s_warp[THREADS / 32];
-  __shared__ Stats s_all[kMaxCluster];
+                                                        float eps, unsigned int* err) {
   __shared__ float s_a[kMaxGroupChannels], s_b[kMaxGroupChannels];
+  __shared__ float4 s_part[kMaxCluster * (THREADS / 32)];
+  __shared__ uint64_t s_bar;
+  cg::cluster_group cluster = cg::this_cluster();
+  // Shared memory only, so it may overlap the previous kernel: arm the barrier that counts the
+  // cluster's cs x nw incoming triples, then tell the peers it is armed.
+  if (threadIdx.x == 0)
+    bar_init_expect(smem_addr(&s_bar), static_cast<uint32_t>(cluster.num_blocks() * (THREADS / 32) * sizeof(float4)));
+  cluster_arrive_release();
   sd::grid_dep_wait();
   sd::grid_dep_launch();
-  cg::cluster_group cluster = cg::this_cluster();
   const int rank = static_cast<int>(cluster.block_rank());
   const int64_t grp = blockIdx.x / cluster.num_blocks();  // b * groups + g
   const int g = static_cast<int>(grp % groups);
@@ -270,7 +321,7 @@ __global__ void __launch_bounds__(THREADS, gn_min_blocks(ITEMS, THREADS)) gn_res
       st.m2 += a * a + b * b + c * c + d * d;
     }
   }
-  cluster_group_affine(st, eps, cpg, s_a, s_b, s_warp, s_all);
+  cluster_group_affine_async<THREADS / 32>(st, eps, cpg, s_a, s_b, s_part, smem_addr(&s_bar), err);
 
   const int64_t base4 = base >> 2;  // base is a multiple of 4 (chunk and group_elems are)
   // Channel (within the group) of this thread's item i, element rank * chunk + 4 (tid + i THREADS):
@@ -363,8 +414,10 @@ cudaError_t launch_resident(dim3 grid, int cs, cudaStream_t s, const float* x, c
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1 + sd::pdl_attr(&attr[1]);
+  unsigned int* err = sd::device_status_word();
+  if (!err) return cudaErrorUnknown;
   return cudaLaunchKernelEx(&cfg, gn_resident<ITEMS, THREADS, EPI>, x, gamma, beta, y, group_elems, chunk, hw, cpg,
-                            groups, eps);
+                            groups, eps, err);
 }
 
 // One GroupNorm launch with epilogue EPI; `name` prefixes error messages.
