@@ -37,7 +37,10 @@ def test_workload_shapes(cuda, wid, label, shape):
                                           # channels per group staged in shared memory: 48, 96 and the
                                           # limit 128 (resident path); 160 and 256 take the streaming path
                                           ((1, 48, 32, 32), 1), ((2, 96, 16, 16), 1), ((1, 128, 8, 8), 1),
-                                          ((2, 640, 4, 4), 4), ((1, 256, 8, 8), 1)])
+                                          ((2, 640, 4, 4), 4), ((1, 256, 8, 8), 1),
+                                          # clusters of 8 CTAs x 256 threads with 12 and 10 float4 per
+                                          # thread (the cluster-barrier exchange)
+                                          ((2, 320, 96, 96), 32), ((1, 640, 64, 64), 32)])
 def test_odd_shapes(cuda, shape, groups):
     x = si.normal(shape, 500 + sum(shape))
     C = shape[1]

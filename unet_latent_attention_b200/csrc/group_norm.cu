@@ -9,11 +9,12 @@
 //    streaming loads, so HBM is read exactly once (the resident path).
 //  * Statistics stay in fp32 but are merged as (count, mean, M2) triples with the pairwise update
 //    of Chan, Golub and LeVeque (1979) instead of sum / sum-of-squares, which cancels when
-//    |mean| >> std. Resident path: warp shuffles, then every warp sends its triple into every
-//    cluster peer's shared memory with st.async, counted on the peer's mbarrier (no cluster-wide
-//    barrier on the critical path); streaming path: shared memory across warps, then distributed
-//    shared memory across the cluster behind one cluster barrier. Every CTA of a cluster merges
-//    the triples in one fixed order, so all of them obtain bit-identical statistics.
+//    |mean| >> std. Resident path with clusters of up to 4 CTAs: warp shuffles, then every warp
+//    sends its triple into every cluster peer's shared memory with st.async, counted on the peer's
+//    mbarrier (no cluster-wide barrier on the critical path); clusters of 8 and the streaming
+//    path: shared memory across warps, then one push per CTA into distributed shared memory behind
+//    one cluster barrier. Every CTA of a cluster merges the triples in one fixed order, so all of
+//    them obtain bit-identical statistics.
 //  * The tail is fused: y = x * a_c + b_c with a_c = rstd * gamma[c], b_c = beta[c] - mean * a_c.
 //    sd_group_norm_silu adds the SiLU activation, v * sigmoid(v), that follows GroupNorm in the
 //    UNet's residual blocks (the page's GroupNorm + SiLU single-kernel fusion, §9), with an fp32 or
@@ -216,6 +217,43 @@ __device__ __forceinline__ void cluster_group_stats(Stats st, float eps, float* 
   __syncthreads();
 }
 
+// Resident path's statistics, then the per-channel affine of the group: the thread's triple is
+// merged over its warp (shuffles), the warps' triples by warp 0 (one shuffle tree), and warp 0's
+// lanes push the CTA's triple into slot `rank` of every peer's shared memory at once; after one
+// cluster barrier warp 0 merges the slots in a fixed tree (so every CTA of the cluster obtains the
+// same bits) and writes a_c = rstd * gamma_c and b_c = beta_c - mean * a_c for the group's cpg
+// channels (gamma and beta already staged in s_a / s_b) into shared memory.
+__device__ __forceinline__ void cluster_group_affine(Stats st, float eps, int cpg, float* s_a, float* s_b,
+                                                     Stats* s_warp, Stats* s_all) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const Stats o = shfl_down(st, off);
+    if (lane + off < 32) st = merge_fast(st, o);
+  }
+  if (lane == 0) s_warp[warp] = st;
+  __syncthreads();
+  const int cs = static_cast<int>(cluster.num_blocks());
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;  // 8, 16 or 32
+    const Stats a = warp_tree_merge(lane < nw ? s_warp[lane] : Stats{0.f, 0.f, 0.f}, nw);
+    if (lane < cs) *cluster.map_shared_rank(&s_all[cluster.block_rank()], lane) = a;
+  }
+  cluster.sync();  // release/acquire: every peer's slot write is visible
+  if (warp == 0) {
+    const Stats a = warp_tree_merge(lane < cs ? s_all[lane] : Stats{0.f, 0.f, 0.f}, cs);
+    const float var = a.n > 0.f ? fmaxf(a.m2 / a.n, 0.f) : 0.f;
+    const float rstd = rsqrtf(var + eps);
+    for (int c = lane; c < cpg; c += 32) {
+      const float ac = rstd * s_a[c];
+      s_b[c] = fmaf(-a.mean, ac, s_b[c]);
+      s_a[c] = ac;
+    }
+  }
+  __syncthreads();
+}
+
 // Resident path's statistics without a cluster barrier: each warp merges its threads' triples
 // (shuffles) and sends the warp's triple, by st.async, into slot (rank, warp) of every peer's
 // shared memory, where the bytes complete the peer's mbarrier (armed for cs x nw slots before the
@@ -270,20 +308,27 @@ constexpr int gn_min_blocks(int items, int threads) {
                         : threads == 256 ? (items <= 5 ? 4 : items <= 10 ? 3 : 1) : 1;
 }
 
-template <int ITEMS, int THREADS, int EPI>
+// XCHG selects the statistics exchange: per-warp st.async into every peer (measured faster with
+// clusters of up to 4 CTAs) or one push per CTA and a cluster barrier (faster with clusters of 8:
+// [8,320,96,96] 52.1 -> 47.5 us, [16,320,128,128] 125.6 -> 124.2 us).
+template <int ITEMS, int THREADS, int EPI, bool XCHG>
 __global__ void __launch_bounds__(THREADS, gn_min_blocks(ITEMS, THREADS)) gn_resident(const float* x, const float* __restrict__ gamma,
                                                         const float* __restrict__ beta, void* y,
                                                         int group_elems, int chunk, int hw, int cpg, int groups,
                                                         float eps, unsigned int* err) {
   __shared__ float s_a[kMaxGroupChannels], s_b[kMaxGroupChannels];
-  __shared__ float4 s_part[kMaxCluster * (THREADS / 32)];
+  __shared__ float4 s_part[XCHG ? kMaxCluster * (THREADS / 32) : 1];
+  __shared__ Stats s_warp[XCHG ? 1 : THREADS / 32];
+  __shared__ Stats s_all[XCHG ? 1 : kMaxCluster];
   __shared__ uint64_t s_bar;
   cg::cluster_group cluster = cg::this_cluster();
-  // Shared memory only, so it may overlap the previous kernel: arm the barrier that counts the
-  // cluster's cs x nw incoming triples, then tell the peers it is armed.
-  if (threadIdx.x == 0)
-    bar_init_expect(smem_addr(&s_bar), static_cast<uint32_t>(cluster.num_blocks() * (THREADS / 32) * sizeof(float4)));
-  cluster_arrive_release();
+  if constexpr (XCHG) {
+    // Shared memory only, so it may overlap the previous kernel: arm the barrier that counts the
+    // cluster's cs x nw incoming triples, then tell the peers it is armed.
+    if (threadIdx.x == 0)
+      bar_init_expect(smem_addr(&s_bar), static_cast<uint32_t>(cluster.num_blocks() * (THREADS / 32) * sizeof(float4)));
+    cluster_arrive_release();
+  }
   sd::grid_dep_wait();
   sd::grid_dep_launch();
   const int rank = static_cast<int>(cluster.block_rank());
@@ -321,7 +366,8 @@ __global__ void __launch_bounds__(THREADS, gn_min_blocks(ITEMS, THREADS)) gn_res
       st.m2 += a * a + b * b + c * c + d * d;
     }
   }
-  cluster_group_affine_async<THREADS / 32>(st, eps, cpg, s_a, s_b, s_part, smem_addr(&s_bar), err);
+  if constexpr (XCHG) cluster_group_affine_async<THREADS / 32>(st, eps, cpg, s_a, s_b, s_part, smem_addr(&s_bar), err);
+  else cluster_group_affine(st, eps, cpg, s_a, s_b, s_warp, s_all);
 
   const int64_t base4 = base >> 2;  // base is a multiple of 4 (chunk and group_elems are)
   // Channel (within the group) of this thread's item i, element rank * chunk + 4 (tid + i THREADS):
@@ -416,8 +462,11 @@ cudaError_t launch_resident(dim3 grid, int cs, cudaStream_t s, const float* x, c
   cfg.numAttrs = 1 + sd::pdl_attr(&attr[1]);
   unsigned int* err = sd::device_status_word();
   if (!err) return cudaErrorUnknown;
-  return cudaLaunchKernelEx(&cfg, gn_resident<ITEMS, THREADS, EPI>, x, gamma, beta, y, group_elems, chunk, hw, cpg,
-                            groups, eps, err);
+  if (cs <= 4)
+    return cudaLaunchKernelEx(&cfg, gn_resident<ITEMS, THREADS, EPI, true>, x, gamma, beta, y, group_elems, chunk, hw,
+                              cpg, groups, eps, err);
+  return cudaLaunchKernelEx(&cfg, gn_resident<ITEMS, THREADS, EPI, false>, x, gamma, beta, y, group_elems, chunk, hw,
+                            cpg, groups, eps, err);
 }
 
 // One GroupNorm launch with epilogue EPI; `name` prefixes error messages.
