@@ -62,7 +62,9 @@ typedef enum sd_status {
  * 262144 elements and at most 128 channels, with H*W % 4 == 0 and 16-byte aligned x and y, are
  * read from HBM once (a thread-block cluster of up to 8 CTAs holds the group in registers); other
  * shapes take a streaming path of the same single launch that reads x twice. No global scratch
- * is used.
+ * is used. The CTAs of a cluster exchange their partial statistics through distributed shared
+ * memory; the wait for the peers' triples is bounded (about a second): should it expire, the
+ * output is undefined and sd_device_status() reports SD_ERR_TIMEOUT.
  */
 sd_status sd_group_norm(const float* x, const float* gamma, const float* beta, float* y,
                         int64_t B, int64_t C, int64_t H, int64_t W, int64_t groups, float eps,
