@@ -258,9 +258,9 @@ sd_status sd_debug_attention_ranges(int64_t items, int64_t nkv, int64_t grid, in
  * any device) skip loading its first V tile, so each CTA's bounded wait expires after about one
  * second, the CTA drains its own copies, frees its tensor memory and returns, and
  * sd_device_status() reports SD_ERR_TIMEOUT. Outputs of such launches are undefined. Bit 1 holds
- * back the tail piece of every item split between two CTAs by about 50 us, so that the head piece
- * finishes first and the tail piece merges (the results are unchanged). flags = 0 restores normal
- * operation. Not for production use.
+ * back the tail piece of every item split between two CTAs by about 50 us before it claims the
+ * hand-off slot, so that the head piece claims and publishes and the tail piece merges (the
+ * results are unchanged). flags = 0 restores normal operation. Not for production use.
  */
 void sd_debug_set_fault(int flags);
 
