@@ -231,7 +231,7 @@ struct Bars {
   __device__ uint32_t fin() const { return base + 8 * (2 + 4 * stages + 4 * nq); }
   __device__ uint32_t tok(int t, int q) const { return base + 8 * (2 + 4 * stages + 5 * nq + 4 * t + q); }
   __device__ uint32_t q_empty(int b) const { return base + 8 * (2 + 4 * stages + 5 * nq + 8 + b); }
-  // split-item hand-off of the tail piece (kind 0) and the head piece (kind 1): the leader's
+  // split-item hand-off of the tail piece (kind 0) and the head piece (kind 1): the MMA issuer's
   // decision is published, and this piece's slot has been written by every softmax thread
   __device__ uint32_t split_dec(int kind) const { return base + 8 * (2 + 4 * stages + 5 * nq + 10 + kind); }
   __device__ uint32_t split_written(int kind) const { return base + 8 * (2 + 4 * stages + 5 * nq + 12 + kind); }
@@ -756,7 +756,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       float* slot = ws + static_cast<size_t>(bnd) * C::SLOT_FLOATS;
       unsigned int* cnt = flags + bnd;
       volatile int* dec = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 8) + kind;
-      const bool leader_warp = warp == C::SOFT_WARP0 + 4 * NQ - 1;  // completes a publication
+      const bool leader_warp = warp == C::SOFT_WARP0 + 4 * NQ - 1;  // completes a publication, resets after a merge
       __syncwarp();
       if (!__all_sync(0xffffffffu, wait_bar(bars.split_dec(kind), 0, abort_flag, err)) || *dec == kSplitAbort) {
         ok = false;
