@@ -75,3 +75,18 @@ def test_sdxl_top_level_groups(cuda, B):
     x, gamma, beta = si.group_norm_inputs(4, shape, sub=11 + B)
     y = _gn(x, gamma, beta, 32, 1e-5, cuda)
     assert rel_err(y, oracle.group_norm(x, gamma, beta, 32, 1e-5)) <= REL
+
+
+@pytest.mark.parametrize("shape", [(2, 320, 64, 64), (2, 320, 96, 96), (2, 1280, 16, 16)])
+def test_repeated_launches_are_bit_identical(cuda, shape):
+    # Every CTA of a cluster merges the exchanged statistics in one fixed order, so the output does
+    # not depend on which CTA finished first: clusters of 4 x 512 (st.async exchange), 8 x 256
+    # (cluster-barrier exchange) and 4 x 256 threads.
+    x = torch.from_numpy(si.normal(shape, 900 + shape[1])).to(cuda)
+    C = shape[1]
+    gamma = torch.from_numpy((1 + 0.1 * si.normal((C,), 901)).astype(np.float32)).to(cuda)
+    beta = torch.from_numpy((0.1 * si.normal((C,), 902)).astype(np.float32)).to(cuda)
+    ys = [sdk.sd_group_norm(x, gamma, beta, 32, 1e-5) for _ in range(4)]
+    sdk.sd_device_status()
+    for y in ys[1:]:
+        assert torch.equal(y, ys[0])
