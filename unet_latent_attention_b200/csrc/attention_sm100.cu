@@ -647,7 +647,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       const float neg_m = -m_run;
       uint32_t pk[BN / 2];
-      float ls0 = 0.f, ls1 = 0.f;
+      float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
       // Exponentials in blocks of EB column pairs: all arguments, then all exp2 (special-function
       // unit, or the FMA-pipe polynomial for POLY_PAIRS of every 8 pairs), then all packing, so
       // that a warp keeps many independent exp2 in flight instead of waiting on each pair.
@@ -677,7 +677,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
 #pragma unroll
         for (int i = 0; i < EB; ++i) {
-          if constexpr (!C::L_IN_V) add2(ls0, ls1, ls0, ls1, x[2 * i], x[2 * i + 1]);
+          if constexpr (!C::L_IN_V) {  // fp32 row sums in two chains of pairs (half the dependent adds)
+            if ((b + i) & 1) add2(ls2, ls3, ls2, ls3, x[2 * i], x[2 * i + 1]);
+            else add2(ls0, ls1, ls0, ls1, x[2 * i], x[2 * i + 1]);
+          }
           pk[b + i] = C::F16 ? pack_f16x2(x[2 * i], x[2 * i + 1]) : pack_bf16x2(x[2 * i], x[2 * i + 1]);
         }
         if (kChunkP && (b + EB) % 16 == 0) {  // 16 packed columns done: store them now
@@ -688,7 +691,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tmem_st16(tP + c * 16, r);
         }
       }
-      if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, ls0 + ls1);
+      if constexpr (!C::L_IN_V) l_run = fmaf(l_run, alpha, (ls0 + ls1) + (ls2 + ls3));
       if (kPing && kRelease == BN / 2) {
         __syncwarp();
         if (lane == 0) mbar_arrive(bars.tok(1 - t, quarter));
